@@ -19,7 +19,8 @@
  *           amax == 0 -> 1; a non-finite result -> FLT_MAX
  *   per block: s = (a_b / 6) * S_enc  (two fp32 round-to-nearest ops)
  *              sf = E4M3(s), round to nearest, ties to even, saturating
- *              inv = (sf == 0) ? 0 : S_enc / sf
+ *              inv = (sf == 0) ? 0 : S_enc / sf, clamped to FLT_MAX if it
+ *                    overflows (tensors with amax below ~1e-35)
  *              q_i = E2M1(x_i * inv), round to nearest even, saturating,
  *                    sign kept (a negative value that rounds to 0 is -0)
  *   packing: byte j of a row holds element 2j in the low nibble
@@ -172,6 +173,7 @@ static uint8_t quantize_block(const float *x, float s_enc, uint8_t *codes)
     uint8_t sf = ref_e4m3_encode(s);
     float sfv = (float)ref_e4m3_value(sf);
     float inv = (sfv == 0.0f) ? 0.0f : s_enc / sfv;
+    if (!isfinite(inv)) inv = FLT_MAX;   /* only when S_enc is near FLT_MAX */
     for (int i = 0; i < 16; i++) codes[i] = ref_e2m1_encode(x[i] * inv);
     return sf;
 }

@@ -208,5 +208,10 @@ def test_bf16_subnormal_tensor(orc):
     # that is ~0.041666 = 1.333 * 2^-5, between 1.25 and 1.375 (midpoint
     # 1.3125) -> mantissa 3, exponent field 2 -> code 0x13.
     assert sf[0] == 0x13
-    # inv = FLT_MAX / 0.04296875 overflows to inf; x * inv saturates to +-6.
-    assert np.all((q & 0x7) == 0x7) and np.all(((q >> 4) & 0x7) == 0x7)
+    # inv = FLT_MAX / 0.04296875 overflows and is clamped to FLT_MAX, so
+    # x * inv = 2^-130 * FLT_MAX = 0.25 * (1 - 2^-24) -> below the 0|0.5 tie -> 0
+    # (with the sign kept); a zero element stays 0 instead of becoming NaN.
+    assert np.all(q == 0x80)
+    z = _bits(np.array([tiny, 0.0] * 8, dtype=np.float32))
+    qz, _ = orc.quantize(z, 1, 16, s_enc)
+    assert np.all(qz == 0)
