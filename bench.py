@@ -1,0 +1,420 @@
+"""Benchmark of the NVFP4 linear-layer hot path on B200.
+
+One step = one pass of the whole per-call path over one batch of synthetic
+DiT activations: for every layer of the workload, the per-tensor amax, the
+dynamic NVFP4 quantize and the block-scaled FP4 GEMM (with the fused
+next-layer quantize where the layer feeds one).  Weights are quantized once,
+before timing (static scale).  The headline metric is NVFP4 GEMM TFLOP/s
+including the activation quantize, i.e. 2*M*N*K / (t_amax + t_quantize +
+t_gemm) summed over layers.
+
+Multi-GPU: one process per GPU (torchrun); each rank runs an independent
+replica of the workload (the linear layer needs no exchange), so scaling is
+weak and the value is the work of all ranks over the max-over-ranks time.
+
+--impl reference times the CPU oracle (test infrastructure, the only
+reference for this path) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, layer_inputs  # noqa: E402
+
+METRIC = "NVFP4 GEMM TFLOPS incl. act quantize (% FP4 peak); quantize GB/s (% HBM)"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "qkv_1024"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_PER_BF16 = 4.0      # nominal dense FP4 / dense BF16 (9 / 2.25 PFLOP/s)
+NOMINAL_FP4_TFLOPS = 9000.0
+
+
+def load_peaks() -> tuple[dict, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- distributed plumbing
+
+def dist_env() -> tuple[int, int, int]:
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device) -> None:
+    if dist is not None:
+        t = torch.zeros(1, device=device)
+        dist.all_reduce(t)
+
+
+def aggregate(per_rank_units: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: units processed by all ranks / max-over-ranks time."""
+    return per_rank_units * world / max_seconds
+
+
+# ----------------------------------------------------------------- clocks
+
+CLOCK_FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+                "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+                "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons (read-only)."""
+
+    def __init__(self, index: int, period_ms: int = 50):
+        self.samples: list[tuple[float, list[str]]] = []
+        self.proc = None
+        self.index = index
+        self.period_ms = period_ms
+        self.window: tuple[float, float] | None = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={','.join(CLOCK_FIELDS)}",
+                 "--format=csv,noheader,nounits", f"-lms={self.period_ms}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == len(CLOCK_FIELDS):
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = self.samples
+        if self.window is not None:
+            lo, hi = self.window
+            inside = [r for r in rows if lo - 0.06 <= r[0] <= hi + 0.06]
+            rows = inside if inside else rows
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1][0]) for r in rows if r[1][0].replace(".", "").isdigit()]
+        mx = [float(r[1][1]) for r in rows if r[1][1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[1][4:8]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows),
+                "power_w_max": max((float(r[1][2]) for r in rows
+                                    if r[1][2].replace(".", "").isdigit()), default=None)}
+
+
+# ----------------------------------------------------------------- the GPU arm
+
+class Layer:
+    def __init__(self, nv, spec, x_cpu, w_cpu, device):
+        self.spec = spec
+        self.M, self.K = x_cpu.shape
+        self.N = w_cpu.shape[0]
+        self.x = x_cpu.to(device)
+        self.x_cpu = x_cpu
+        self.lin = nv.NVFP4Linear(w_cpu.to(device))
+        self.xq = nv.empty_nvfp4(self.M, self.K, device)
+        self.amax = torch.empty(1, dtype=torch.float32, device=device)
+        self.y = torch.empty(self.M, self.N, dtype=torch.bfloat16, device=device)
+        self.fused = None
+        if spec.fused_out:
+            # Next-layer tensor scale: static, from a calibration amax of 8.
+            self.fused = nv.FusedQuant(torch.tensor([2688.0 / 8.0], device=device),
+                                       nv.empty_nvfp4(self.M, self.N, device),
+                                       torch.empty(1, dtype=torch.float32, device=device))
+
+    @property
+    def flops(self) -> int:
+        return 2 * self.M * self.N * self.K
+
+    @property
+    def quant_bytes(self) -> int:
+        """Algorithmic bytes of amax (read X) + quantize (read X, write codes + scales)."""
+        import nvfp4_block_scaled_19_b200 as nv
+        n = self.M * self.K
+        return 2 * n + 2 * n + n // 2 + nv.sf_bytes(self.M, self.K)
+
+
+def run_step(nv, layers, ev=None):
+    """One pass of the hot path; ev: optional per-layer event pairs around the
+    quantize pair and the GEMM."""
+    for i, L in enumerate(layers):
+        if ev is not None:
+            ev[i][0].record()
+        nv.tensor_amax(L.x, L.amax)
+        nv.quantize(L.x, L.amax, L.xq)
+        if ev is not None:
+            ev[i][1].record()
+        nv.gemm(L.xq, L.lin.w, L.y, L.fused)
+        if ev is not None:
+            ev[i][2].record()
+
+
+def gpu_arm(args) -> dict | None:
+    import nvfp4_block_scaled_19_b200 as nv
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    nv.lib()
+    peaks, peak_src = load_peaks()
+    w = WORKLOADS[args.workload]
+    layers = [Layer(nv, l, *layer_inputs(w, i), device) for i, l in enumerate(w.layers)]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        run_step(nv, layers)
+    torch.cuda.synchronize()
+    code, detail = nv.device_error()
+    if code != 0:
+        raise RuntimeError(f"device wait timed out during warm-up (tag {detail})")
+
+    n_l = len(layers)
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_l)]
+          for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for s in range(args.steps):
+        flush.zero_()          # L2 flush between steps, outside the timed spans
+        run_step(nv, layers, ev[s])
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(dist, device)
+    time.sleep(0.1)
+    sampler.window = (t_wall0, t_wall1)
+    sampler.stop()
+    code, detail = nv.device_error()
+    if code != 0:
+        raise RuntimeError(f"device wait timed out (tag {detail})")
+
+    q_ms = [[ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)] for i in range(n_l)]
+    g_ms = [[ev[s][i][1].elapsed_time(ev[s][i][2]) for s in range(args.steps)] for i in range(n_l)]
+    step_ms = [sum(q_ms[i][s] + g_ms[i][s] for i in range(n_l)) for s in range(args.steps)]
+    total_s = sum(step_ms) / 1e3
+    total_s = max_over_ranks(total_s, dist, device)
+    flops_step = sum(L.flops for L in layers)
+    value = aggregate(flops_step * args.steps, world, total_s) / 1e12
+
+    # Roofline of the dominant kernel (the GEMM), live CUDA-event durations.
+    g_avg = [sum(g) / len(g) for g in g_ms]
+    q_avg = [sum(q) / len(q) for q in q_ms]
+    top = max(range(n_l), key=lambda i: g_avg[i])
+    bf16_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    bf16_sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    fp4_peak = FP4_PER_BF16 * bf16_burst
+    gemm_tflops = layers[top].flops / (g_avg[top] * 1e-3) / 1e12
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    q_bytes = sum(L.quant_bytes for L in layers)
+    q_gbs = q_bytes / (sum(q_avg) * 1e-3) / 1e9
+
+    e2e = host_e2e(nv, layers, args, device, dist, world)
+    clocks = sampler.summary()
+
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(sum(step_ms) / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x ue4m3 block scales, fp32 accumulate, bf16 out)",
+        "data": "synthetic (seeded DiT-shaped activations and N(0,1/K) weights)",
+        "config": {"workload": w.name, "description": w.description, "M": w.M,
+                   "layers": [[l.name, l.K, l.N] for l in w.layers],
+                   "l2": "flushed between steps (256 MiB write, outside the timed spans)",
+                   "parallelism": f"replicas x{world}"},
+        "pct_fp4_peak": {"of_4x_measured_bf16_burst": round(value / world / fp4_peak, 4),
+                         "of_nominal_9pf": round(value / world / NOMINAL_FP4_TFLOPS, 4)},
+        "quantize": {"gbs": round(q_gbs, 1), "pct_hbm": round(q_gbs / hbm, 4),
+                     "ms_per_step": round(sum(q_avg), 5),
+                     "note": "amax + dynamic quantize of every layer input; "
+                             "algorithmic bytes 4.5625 B/elem + scales"},
+        "gemm": {"tflops": round(gemm_tflops, 1), "ms": round(g_avg[top], 5),
+                 "layer": layers[top].spec.name},
+        "roofline": {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 mxf4nvf4)",
+                     "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
+                     "traffic": None,
+                     "peak_source": f"{peak_src}: 4 x bf16_tflops burst ({bf16_burst}); "
+                                    f"sustained would be {FP4_PER_BF16 * bf16_sust}"},
+        "clocks": clocks,
+        "e2e": e2e,
+        "gpu_launches": 3 * n_l * args.steps,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_rows)
+    return line
+
+
+def host_e2e(nv, layers, args, device, dist, world) -> dict:
+    """Same metric through nvfp4_linear_host: pinned host X in, host Y out."""
+    stream = torch.cuda.current_stream()
+    hosts = []
+    for L in layers:
+        xh = L.x_cpu.contiguous().pin_memory()
+        yh = torch.empty(L.M, L.N, dtype=torch.bfloat16).pin_memory()
+        hosts.append((xh, yh, L.lin.host_workspace(L.M, device)))
+    steps = max(1, min(args.steps, args.e2e_steps))
+    for _ in range(2):
+        for L, (xh, yh, ws) in zip(layers, hosts):
+            L.lin.forward_host(xh, yh, ws)
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        for L, (xh, yh, ws) in zip(layers, hosts):
+            L.lin.forward_host(xh, yh, ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    sec = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, device)
+    flops = sum(L.flops for L in layers) * steps
+    return {"value": round(aggregate(flops, world, sec) / 1e12, 3), "unit": UNIT,
+            "h2d_bytes_per_step": sum(L.M * L.K * 2 for L in layers),
+            "d2h_bytes_per_step": sum(L.M * L.N * 2 for L in layers),
+            "steps": steps, "api": "nvfp4_linear_host (C ABI, pinned host buffers)"}
+
+
+# ----------------------------------------------------------------- CPU oracle (baseline / reference)
+
+def oracle_sample(w, rows: int) -> tuple[float, int, str]:
+    """One bounded oracle pass: for every layer, amax + quantize of a `rows`-row
+    slice of X, quantize of W (its static scale), and the dequantize-then-fp64
+    GEMM of that slice. Returns (seconds, flops, description)."""
+    import oracle
+    from workloads import bf16_bits
+    secs, flops = 0.0, 0
+    for li, l in enumerate(w.layers):
+        x, wt = layer_inputs(w, li, M=rows)
+        xb, wb = bf16_bits(x), bf16_bits(wt)
+        bq, bsf, bsd, _ = oracle.quantize_dynamic(wb, l.N, l.K)   # static weights: untimed
+        t0 = time.perf_counter()
+        aq, asf, asd, _ = oracle.quantize_dynamic(xb, rows, l.K)
+        oracle.gemm(aq, asf, asd, bq, bsf, bsd, rows, l.N, l.K)
+        secs += time.perf_counter() - t0
+        flops += 2 * rows * l.N * l.K
+    desc = (f"{rows} rows of every layer input of {w.name} (full K, full N): amax + quantize "
+            f"+ dequantize-then-fp64 GEMM; weight quantize untimed (static)")
+    return secs, flops, desc
+
+
+def cpu_baseline(w, rows: int) -> dict:
+    import oracle
+    oracle.lib()
+    oracle_sample(w, min(rows, 64))       # warm-up
+    runs = [oracle_sample(w, rows) for _ in range(3)]
+    secs = statistics.median(r[0] for r in runs)
+    return {"value": round(runs[0][1] / secs / 1e12, 6), "unit": UNIT,
+            "cores": oracle.num_threads(), "kind": "oracle", "sample": runs[0][2],
+            "seconds": round(secs, 3)}
+
+
+def reference_arm(args) -> dict | None:
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    oracle.lib()
+    w = WORKLOADS[args.workload]
+    for _ in range(max(args.warmup, 1)):
+        oracle_sample(w, min(args.cpu_rows, 64))
+    secs, flops = 0.0, 0
+    desc = ""
+    steps = max(1, args.steps if args.steps <= 20 else 20)
+    for _ in range(steps):
+        s, f, desc = oracle_sample(w, args.cpu_rows)
+        secs += s
+        flops += f
+    value = flops / secs / 1e12
+    cores = oracle.num_threads()
+    return {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "impl": "reference",
+            "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 1),
+            "ms_per_step": round(secs / steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+            "data": "synthetic", "config": {"workload": w.name, "M": w.M,
+                                            "layers": [[l.name, l.K, l.N] for l in w.layers]},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    line = reference_arm(args) if args.impl == "reference" else gpu_arm(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    rank, world, _ = dist_env()
+    if world > 1 and args.impl != "reference":
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,172 @@
+/*
+ * nvfp4.h — C ABI of the B200 (sm_100a) NVFP4 linear-layer library.
+ *
+ * NVFP4 is two-level microblock quantization: an FP32 scale per tensor
+ * (static or dynamic) and a scale per block of 16 elements computed
+ * dynamically ("英伟达B200狂飙10.2倍！AI绘图告别龟速！", section
+ * "NVFP4量化：在精度与速度之间寻得最佳平衡"; "Scaling NVFP4 Inference for
+ * FLUX.2 on NVIDIA Blackwell Data Center GPUs", section "Key Questions
+ * Answered").  Encoding used here: E2M1 elements (two per byte, the even
+ * element in the low nibble) and unsigned E4M3 block scales.
+ *
+ * Quantization of a bf16 tensor X[rows, cols] (cols % 16 == 0), blocks of 16
+ * contiguous elements along cols:
+ *   S_enc = 2688 / amax        (1 if amax == 0, FLT_MAX if not finite)
+ *   S_dec = 1 / S_enc
+ *   per block b:  sf_b = E4M3_rn_satfinite((max|x| / 6) * S_enc)
+ *                 q_i  = E2M1_rn_satfinite(x_i * (S_enc / sf_b)), 0 if sf_b == 0
+ * Every fp32 step is one IEEE round-to-nearest-even operation, so results are
+ * bit-reproducible.  A negative value that rounds to zero keeps its sign (-0).
+ *
+ * Scale-factor layout ("tiled SF"): pad128(rows) x pad4(cols/16) bytes in
+ * 128-row x 4-block tiles of 512 bytes, tiles ordered row-block-major; in a
+ * tile, (r, c) is at byte (r%32)*16 + ((r/32)%4)*4 + c%4.  Padding bytes are
+ * written as 0.  This is the layout the tcgen05 block-scaled MMA consumes.
+ *
+ * GEMM: Y[m,n] = bf16_rn( a_s_dec * b_s_dec *
+ *                sum_k e2m1(Aq[m,k]) sfA[m,k/16] e2m1(Bq[n,k]) sfB[n,k/16] )
+ * with A = activations [M,K] and B = weights [N,K] (nn.Linear layout), fp32
+ * accumulation in tensor memory.
+ *
+ * Conventions for every call below:
+ *  - Pointers marked "device" are device memory owned by the caller; the
+ *    library never allocates, frees or synchronises, and keeps no pointer
+ *    after the call returns.  "host" pointers are host memory (pinned for
+ *    truly asynchronous copies).
+ *  - Work is enqueued on `stream` (NULL = legacy default stream) and runs
+ *    asynchronously; results are valid after the stream is synchronised.
+ *  - Argument errors are returned synchronously before anything is
+ *    enqueued; launch errors are returned as NVFP4_ERR_LAUNCH.  Nothing
+ *    aborts or throws across the ABI.  A kernel that gives up on a bounded
+ *    wait records NVFP4_ERR_TIMEOUT in a device word read by
+ *    nvfp4_device_error().
+ *  - Device pointers must be 16-byte aligned (NVFP4_ERR_MISALIGNED).
+ *  - The device must be sm_100 (B200); otherwise NVFP4_ERR_UNSUPPORTED_DEVICE.
+ *  - Inputs must be finite (no NaN/inf in X or W).
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st *nvfp4_stream_t;
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARG = 1,
+    NVFP4_ERR_MISALIGNED = 2,
+    NVFP4_ERR_UNSUPPORTED_DEVICE = 3,
+    NVFP4_ERR_LAUNCH = 4,
+    NVFP4_ERR_TIMEOUT = 5
+} nvfp4_status;
+
+/* Optional fused output quantization of the GEMM (the next layer's
+ * activation quantize, done in the GEMM epilogue).  Y is first rounded to
+ * bf16, then quantized in blocks of 16 along N with the caller's S_enc
+ * (static, or the previous call's amax via 2688/amax).  Requires N % 16 == 0.
+ *   s_enc_y  device, 1 fp32, read
+ *   yq       device, M*N/2 bytes, written (packed E2M1, row-major)
+ *   ysf      device, nvfp4_sf_bytes(M, N) bytes, written (tiled SF, padding 0)
+ *   amax_y   device, 1 fp32, overwritten with max|Y| over the bf16 Y
+ *            (NULL = not computed). */
+typedef struct {
+    const float *s_enc_y;
+    uint8_t *yq;
+    uint8_t *ysf;
+    float *amax_y;
+} nvfp4_fused_out;
+
+/* Bytes of packed E2M1 data for a [rows, cols] tensor: rows * cols / 2. */
+size_t nvfp4_packed_bytes(int64_t rows, int64_t cols);
+
+/* Bytes of the tiled scale-factor buffer: pad128(rows) * pad4(cols / 16). */
+size_t nvfp4_sf_bytes(int64_t rows, int64_t cols);
+
+/* Static description of a status code (never NULL). */
+const char *nvfp4_status_string(nvfp4_status status);
+
+/* Per-tensor absolute maximum, the input of the dynamic per-tensor scale
+ * (FP32 per-tensor scale "computed statically or dynamically": nmedialink
+ * page above, NVFP4 section).
+ *   x_bf16    device, numel bf16 values, read
+ *   numel     >= 0 (0 writes amax = 0)
+ *   amax_dev  device, 1 fp32, overwritten with max_i |x_i| */
+nvfp4_status nvfp4_tensor_amax(const void *x_bf16, int64_t numel, float *amax_dev,
+                               nvfp4_stream_t stream);
+
+/* Dynamic NVFP4 quantization (per-16 block scales computed at run time:
+ * nmedialink page above, NVFP4 section).  S_enc is derived on the device
+ * from *amax_dev, so no host synchronisation is needed.
+ *   x_bf16     device, [rows, cols] row-major bf16, read; cols % 16 == 0
+ *   amax_dev   device, 1 fp32, read (normally from nvfp4_tensor_amax)
+ *   q_out      device, rows*cols/2 bytes, written
+ *   sf_out     device, nvfp4_sf_bytes(rows, cols) bytes, written (incl. padding)
+ *   s_dec_out  device, 1 fp32, written with 1/S_enc (NULL = not written) */
+nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t rows, int64_t cols,
+                            const float *amax_dev, uint8_t *q_out, uint8_t *sf_out,
+                            float *s_dec_out, nvfp4_stream_t stream);
+
+/* Static-scale variant: same as nvfp4_quantize but S_enc is given directly
+ * (the per-tensor scale "computed statically": nmedialink page above).
+ *   s_enc_dev  device, 1 fp32 > 0, read */
+nvfp4_status nvfp4_quantize_with_scale(const void *x_bf16, int64_t rows, int64_t cols,
+                                       const float *s_enc_dev, uint8_t *q_out,
+                                       uint8_t *sf_out, float *s_dec_out,
+                                       nvfp4_stream_t stream);
+
+/* Block-scaled FP4 GEMM on tcgen05 tensor cores, Y = X . W^T (the NVFP4
+ * linear layer whose weights are quantized once, "quantize_weights=True",
+ * nmedialink page above, NVFP4 section).
+ *   aq, asf, a_s_dec   device: activations [M,K] quantized (packed, tiled SF,
+ *                      1 fp32 decode scale)
+ *   bq, bsf, b_s_dec   device: weights [N,K] quantized likewise
+ *   M >= 1, N >= 1 with N % 8 == 0, K >= 64 with K % 64 == 0
+ *   y_bf16             device, [M,N] row-major bf16, written (NULL allowed
+ *                      only when fused != NULL)
+ *   fused              NULL, or the fused output quantization above */
+nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_dec,
+                        const uint8_t *bq, const uint8_t *bsf, const float *b_s_dec,
+                        int64_t M, int64_t N, int64_t K, void *y_bf16,
+                        const nvfp4_fused_out *fused, nvfp4_stream_t stream);
+
+/* Device buffers for nvfp4_linear_host (all caller-owned device memory):
+ *   x      [M,K] bf16      xq  M*K/2 bytes      xsf  nvfp4_sf_bytes(M,K)
+ *   amax   1 fp32          s_dec 1 fp32         y    [M,N] bf16 */
+typedef struct {
+    void *x;
+    uint8_t *xq;
+    uint8_t *xsf;
+    float *amax;
+    float *s_dec;
+    void *y;
+} nvfp4_linear_workspace;
+
+/* One NVFP4 linear layer from host memory: copies X host->device, runs
+ * amax, dynamic quantize and the GEMM against pre-quantized weights, and
+ * copies Y device->host, all enqueued on `stream` (the per-call activation
+ * path of the pages' NVFP4 linear: dynamic activation quantization, static
+ * weights).
+ *   x_host_bf16   host, [M,K] bf16, read
+ *   wq, wsf, w_s_dec  device, weights [N,K] quantized once
+ *   y_host_bf16   host, [M,N] bf16, written once the stream completes */
+nvfp4_status nvfp4_linear_host(const void *x_host_bf16, int64_t M, int64_t K,
+                               const uint8_t *wq, const uint8_t *wsf,
+                               const float *w_s_dec, int64_t N, void *y_host_bf16,
+                               const nvfp4_linear_workspace *ws, nvfp4_stream_t stream);
+
+/* Reads and clears the device-side error word of the current device
+ * (synchronises the device).  *code_out = NVFP4_OK or NVFP4_ERR_TIMEOUT;
+ * *detail_out (may be NULL) = which wait gave up (kernel-specific tag). */
+nvfp4_status nvfp4_device_error(int *code_out, int *detail_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

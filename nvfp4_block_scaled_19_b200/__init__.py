@@ -1,0 +1,248 @@
+"""NVFP4 linear layers for B200 (sm_100a): Python binding of libnvfp4.so.
+
+NVFP4 two-level microblock quantization (FP32 per-tensor scale + E4M3 scale
+per 16 elements, E2M1 elements) and the tcgen05 block-scaled FP4 GEMM, as
+used for the linear layers of FLUX diffusion transformers ("英伟达B200狂飙
+10.2倍！AI绘图告别龟速！", section "NVFP4量化"; "Scaling NVFP4 Inference for
+FLUX.2 on NVIDIA Blackwell Data Center GPUs", section "Key Questions
+Answered").
+
+This module only marshals arguments: every step runs in the CUDA kernels of
+libnvfp4.so through its C ABI (include/nvfp4.h).  PyTorch supplies device
+memory and the current stream.  There is no CPU fallback: if the library is
+missing or the device is not sm_100, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "misaligned", 3: "unsupported device",
+          4: "launch error", 5: "device wait timed out"}
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {STATUS.get(status, status)} (status {status})")
+        self.status = status
+
+
+class FusedOut(ctypes.Structure):
+    _fields_ = [("s_enc_y", ctypes.c_void_p), ("yq", ctypes.c_void_p),
+                ("ysf", ctypes.c_void_p), ("amax_y", ctypes.c_void_p)]
+
+
+class LinearWorkspace(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("xq", ctypes.c_void_p), ("xsf", ctypes.c_void_p),
+                ("amax", ctypes.c_void_p), ("s_dec", ctypes.c_void_p), ("y", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C-ABI library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m nvfp4_block_scaled_19_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, st = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.nvfp4_packed_bytes.restype = ctypes.c_size_t
+        L.nvfp4_packed_bytes.argtypes = [i64, i64]
+        L.nvfp4_sf_bytes.restype = ctypes.c_size_t
+        L.nvfp4_sf_bytes.argtypes = [i64, i64]
+        L.nvfp4_status_string.restype = ctypes.c_char_p
+        L.nvfp4_status_string.argtypes = [st]
+        L.nvfp4_tensor_amax.restype = st
+        L.nvfp4_tensor_amax.argtypes = [vp, i64, vp, vp]
+        L.nvfp4_quantize.restype = st
+        L.nvfp4_quantize.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
+        L.nvfp4_quantize_with_scale.restype = st
+        L.nvfp4_quantize_with_scale.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
+        L.nvfp4_gemm.restype = st
+        L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp,
+                                 ctypes.POINTER(FusedOut), vp]
+        L.nvfp4_linear_host.restype = st
+        L.nvfp4_linear_host.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp,
+                                        ctypes.POINTER(LinearWorkspace), vp]
+        L.nvfp4_device_error.restype = st
+        L.nvfp4_device_error.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise NVFP4Error(fn, status)
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def packed_bytes(rows: int, cols: int) -> int:
+    return int(lib().nvfp4_packed_bytes(rows, cols))
+
+
+def sf_bytes(rows: int, cols: int) -> int:
+    return int(lib().nvfp4_sf_bytes(rows, cols))
+
+
+def _require(x: torch.Tensor, dtype, name: str) -> None:
+    if not x.is_cuda or x.dtype != dtype or not x.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+@dataclass
+class NVFP4Tensor:
+    """A quantized [rows, cols] tensor: packed codes, tiled scales, decode scale."""
+    q: torch.Tensor       # uint8 [rows, cols/2]
+    sf: torch.Tensor      # uint8 [sf_bytes(rows, cols)]
+    s_dec: torch.Tensor   # float32 [1] = 1 / S_enc
+    rows: int
+    cols: int
+
+
+def empty_nvfp4(rows: int, cols: int, device=None) -> NVFP4Tensor:
+    dev = torch.device("cuda") if device is None else device
+    return NVFP4Tensor(torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev),
+                       torch.empty(sf_bytes(rows, cols), dtype=torch.uint8, device=dev),
+                       torch.empty(1, dtype=torch.float32, device=dev), rows, cols)
+
+
+def tensor_amax(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """max |x| of a bf16 CUDA tensor into a 1-element fp32 CUDA tensor."""
+    _require(x, torch.bfloat16, "x")
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check("nvfp4_tensor_amax", lib().nvfp4_tensor_amax(x.data_ptr(), x.numel(), out.data_ptr(),
+                                                        _stream(stream)))
+    return out
+
+
+def quantize(x: torch.Tensor, amax: torch.Tensor, out: NVFP4Tensor | None = None,
+             stream=None) -> NVFP4Tensor:
+    """Dynamic NVFP4 quantization of bf16 x[rows, cols] given its amax (device)."""
+    _require(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    out = empty_nvfp4(rows, cols, x.device) if out is None else out
+    _check("nvfp4_quantize", lib().nvfp4_quantize(
+        x.data_ptr(), rows, cols, amax.data_ptr(), out.q.data_ptr(), out.sf.data_ptr(),
+        out.s_dec.data_ptr(), _stream(stream)))
+    return out
+
+
+def quantize_with_scale(x: torch.Tensor, s_enc: torch.Tensor, out: NVFP4Tensor | None = None,
+                        stream=None) -> NVFP4Tensor:
+    """NVFP4 quantization with a static per-tensor scale S_enc (device fp32)."""
+    _require(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    out = empty_nvfp4(rows, cols, x.device) if out is None else out
+    _check("nvfp4_quantize_with_scale", lib().nvfp4_quantize_with_scale(
+        x.data_ptr(), rows, cols, s_enc.data_ptr(), out.q.data_ptr(), out.sf.data_ptr(),
+        out.s_dec.data_ptr(), _stream(stream)))
+    return out
+
+
+def quantize_dynamic(x: torch.Tensor, out: NVFP4Tensor | None = None,
+                     amax: torch.Tensor | None = None, stream=None) -> NVFP4Tensor:
+    """amax then quantize: the per-call activation path."""
+    amax = tensor_amax(x, amax, stream)
+    return quantize(x, amax, out, stream)
+
+
+@dataclass
+class FusedQuant:
+    """Fused next-layer quantization outputs of a GEMM."""
+    s_enc: torch.Tensor           # fp32 [1], read
+    out: NVFP4Tensor              # q [M, N/2], sf tiled; out.s_dec is not written
+    amax: torch.Tensor | None     # fp32 [1], written with max|Y|
+
+
+def gemm(a: NVFP4Tensor, b: NVFP4Tensor, y: torch.Tensor | None = None,
+         fused: FusedQuant | None = None, want_y: bool = True, stream=None) -> torch.Tensor | None:
+    """Y[M,N] = A[M,K] . B[N,K]^T on tcgen05 block-scaled FP4 tensor cores."""
+    M, K = a.rows, a.cols
+    N = b.rows
+    if b.cols != K:
+        raise ValueError("K mismatch")
+    if y is None and want_y:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=a.q.device)
+    fo = None
+    if fused is not None:
+        fo = FusedOut(fused.s_enc.data_ptr(), fused.out.q.data_ptr(), fused.out.sf.data_ptr(),
+                      _ptr(fused.amax))
+    _check("nvfp4_gemm", lib().nvfp4_gemm(
+        a.q.data_ptr(), a.sf.data_ptr(), a.s_dec.data_ptr(), b.q.data_ptr(), b.sf.data_ptr(),
+        b.s_dec.data_ptr(), M, N, K, _ptr(y), ctypes.byref(fo) if fo is not None else None,
+        _stream(stream)))
+    return y
+
+
+class NVFP4Linear:
+    """An nn.Linear-shaped NVFP4 layer: weights quantized once with a static
+    per-tensor scale (from the weight amax, or a given one), activations
+    quantized dynamically on every call."""
+
+    def __init__(self, weight: torch.Tensor, w_amax: torch.Tensor | None = None):
+        _require(weight, torch.bfloat16, "weight")
+        self.N, self.K = weight.shape
+        amax = tensor_amax(weight) if w_amax is None else w_amax
+        self.w = quantize(weight, amax)
+        self._x = None
+
+    def _xbuf(self, M: int, device) -> tuple[NVFP4Tensor, torch.Tensor]:
+        if self._x is None or self._x[0].rows != M:
+            self._x = (empty_nvfp4(M, self.K, device),
+                       torch.empty(1, dtype=torch.float32, device=device))
+        return self._x
+
+    def __call__(self, x: torch.Tensor, y: torch.Tensor | None = None,
+                 fused: FusedQuant | None = None, want_y: bool = True) -> torch.Tensor | None:
+        xq, amax = self._xbuf(x.shape[0], x.device)
+        quantize_dynamic(x, xq, amax)
+        return gemm(xq, self.w, y, fused, want_y)
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, ws: dict,
+                     stream=None) -> None:
+        """Host bf16 X -> host bf16 Y through nvfp4_linear_host (copies included)."""
+        M = x_host.shape[0]
+        w = LinearWorkspace(ws["x"].data_ptr(), ws["xq"].data_ptr(), ws["xsf"].data_ptr(),
+                            ws["amax"].data_ptr(), ws["s_dec"].data_ptr(), ws["y"].data_ptr())
+        _check("nvfp4_linear_host", lib().nvfp4_linear_host(
+            x_host.data_ptr(), M, self.K, self.w.q.data_ptr(), self.w.sf.data_ptr(),
+            self.w.s_dec.data_ptr(), self.N, y_host.data_ptr(), ctypes.byref(w),
+            _stream(stream)))
+
+    def host_workspace(self, M: int, device=None) -> dict:
+        dev = torch.device("cuda") if device is None else device
+        return {"x": torch.empty(M, self.K, dtype=torch.bfloat16, device=dev),
+                "xq": torch.empty(M, self.K // 2, dtype=torch.uint8, device=dev),
+                "xsf": torch.empty(sf_bytes(M, self.K), dtype=torch.uint8, device=dev),
+                "amax": torch.empty(1, dtype=torch.float32, device=dev),
+                "s_dec": torch.empty(1, dtype=torch.float32, device=dev),
+                "y": torch.empty(M, self.N, dtype=torch.bfloat16, device=dev)}
+
+
+def device_error() -> tuple[int, int]:
+    """(code, detail) of the device error word, cleared on read (synchronises)."""
+    c, d = ctypes.c_int(0), ctypes.c_int(0)
+    _check("nvfp4_device_error", lib().nvfp4_device_error(ctypes.byref(c), ctypes.byref(d)))
+    return c.value, d.value
+
+
+def status_string(status: int) -> str:
+    return lib().nvfp4_status_string(status).decode()

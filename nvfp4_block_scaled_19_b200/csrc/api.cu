@@ -1,0 +1,252 @@
+// C ABI of the NVFP4 linear-layer library (declared in include/nvfp4.h):
+// argument checks, device check, TMA descriptor encoding and launches.
+// The library never allocates device memory and never synchronises except in
+// nvfp4_device_error().
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "gemm.h"
+#include "nvfp4.h"
+
+namespace nvfp4 {
+cudaError_t read_and_clear_device_error(int *code, int *detail);
+}
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    int state;  // 0 unknown, 1 supported, 2 unsupported
+    int num_sms;
+};
+DeviceInfo g_devices[kMaxDevices];
+
+nvfp4_status current_device(int *num_sms) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return NVFP4_ERR_UNSUPPORTED_DEVICE;
+    }
+    DeviceInfo &d = g_devices[dev];
+    if (d.state == 0) {
+        int major = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return NVFP4_ERR_UNSUPPORTED_DEVICE;
+        }
+        d.num_sms = sms;
+        d.state = (major == 10) ? 1 : 2;
+    }
+    if (d.state != 1) return NVFP4_ERR_UNSUPPORTED_DEVICE;
+    *num_sms = d.num_sms;
+    return NVFP4_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+nvfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH; }
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// 2-D byte tensor [rows, row_bytes] (row-major), 128-byte-swizzled boxes of
+// box_rows x 128 bytes.
+bool encode_operand_map(CUtensorMap *m, const void *base, uint64_t row_bytes, uint64_t rows,
+                        uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    cuuint64_t dims[2] = {row_bytes, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+nvfp4_status check_quantize_args(const void *x, int64_t rows, int64_t cols, const void *scale,
+                                 const uint8_t *q, const uint8_t *sf) {
+    if (rows < 0 || cols <= 0 || cols % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+    if (rows > (int64_t(1) << 40) / cols) return NVFP4_ERR_INVALID_ARG;
+    if (x == nullptr || scale == nullptr || q == nullptr || sf == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(sf)) return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+nvfp4_status quantize_impl(const void *x, int64_t rows, int64_t cols, const float *scale,
+                           bool dynamic, uint8_t *q, uint8_t *sf, float *s_dec_out,
+                           cudaStream_t stream) {
+    nvfp4_status st = check_quantize_args(x, rows, cols, scale, q, sf);
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    if (rows == 0) return NVFP4_OK;
+    return from_cuda(
+        nvfp4::launch_quantize(x, rows, cols, scale, dynamic, q, sf, s_dec_out, sms, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t nvfp4_packed_bytes(int64_t rows, int64_t cols) {
+    if (rows < 0 || cols < 0) return 0;
+    return static_cast<size_t>(rows) * static_cast<size_t>(cols) / 2;
+}
+
+size_t nvfp4_sf_bytes(int64_t rows, int64_t cols) {
+    if (rows < 0 || cols < 0) return 0;
+    const int64_t kb = cols / 16;
+    return static_cast<size_t>((rows + 127) / 128 * 128) * static_cast<size_t>((kb + 3) / 4 * 4);
+}
+
+const char *nvfp4_status_string(nvfp4_status s) {
+    switch (s) {
+        case NVFP4_OK: return "ok";
+        case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+        case NVFP4_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case NVFP4_ERR_UNSUPPORTED_DEVICE: return "no sm_100 (B200) CUDA device";
+        case NVFP4_ERR_LAUNCH: return "kernel launch or CUDA runtime error";
+        case NVFP4_ERR_TIMEOUT: return "a device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+nvfp4_status nvfp4_tensor_amax(const void *x_bf16, int64_t numel, float *amax_dev,
+                               nvfp4_stream_t stream) {
+    if (numel < 0 || amax_dev == nullptr || (numel > 0 && x_bf16 == nullptr))
+        return NVFP4_ERR_INVALID_ARG;
+    if (numel > 0 && !aligned16(x_bf16)) return NVFP4_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(amax_dev) & 3u) != 0) return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    nvfp4_status st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_amax(x_bf16, numel, amax_dev, sms, stream));
+}
+
+nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t rows, int64_t cols, const float *amax_dev,
+                            uint8_t *q_out, uint8_t *sf_out, float *s_dec_out,
+                            nvfp4_stream_t stream) {
+    return quantize_impl(x_bf16, rows, cols, amax_dev, true, q_out, sf_out, s_dec_out, stream);
+}
+
+nvfp4_status nvfp4_quantize_with_scale(const void *x_bf16, int64_t rows, int64_t cols,
+                                       const float *s_enc_dev, uint8_t *q_out, uint8_t *sf_out,
+                                       float *s_dec_out, nvfp4_stream_t stream) {
+    return quantize_impl(x_bf16, rows, cols, s_enc_dev, false, q_out, sf_out, s_dec_out, stream);
+}
+
+nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_dec,
+                        const uint8_t *bq, const uint8_t *bsf, const float *b_s_dec, int64_t M,
+                        int64_t N, int64_t K, void *y_bf16, const nvfp4_fused_out *fused,
+                        nvfp4_stream_t stream) {
+    if (M < 1 || N < 8 || N % 8 != 0 || K < 64 || K % 64 != 0) return NVFP4_ERR_INVALID_ARG;
+    if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31))
+        return NVFP4_ERR_INVALID_ARG;
+    if (aq == nullptr || asf == nullptr || a_s_dec == nullptr || bq == nullptr ||
+        bsf == nullptr || b_s_dec == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (y_bf16 == nullptr && fused == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (fused != nullptr &&
+        (N % 16 != 0 || fused->s_enc_y == nullptr || fused->yq == nullptr || fused->ysf == nullptr))
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(aq) || !aligned16(bq) || !aligned16(asf) || !aligned16(bsf) ||
+        (y_bf16 != nullptr && !aligned16(y_bf16)))
+        return NVFP4_ERR_MISALIGNED;
+    if (fused != nullptr && (!aligned16(fused->yq) || !aligned16(fused->ysf)))
+        return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    nvfp4_status st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+
+    const int tile_n = nvfp4::gemm_tile_n(M, N);
+    CUtensorMap ta, tb;
+    std::memset(&ta, 0, sizeof(ta));
+    std::memset(&tb, 0, sizeof(tb));
+    if (!encode_operand_map(&ta, aq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M), 128) ||
+        !encode_operand_map(&tb, bq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N),
+                            static_cast<uint32_t>(tile_n)))
+        return NVFP4_ERR_LAUNCH;
+
+    nvfp4::GemmParams p;
+    p.asf = asf;
+    p.bsf = bsf;
+    p.a_s_dec = a_s_dec;
+    p.b_s_dec = b_s_dec;
+    p.y = static_cast<uint8_t *>(y_bf16);
+    p.s_enc_y = fused ? fused->s_enc_y : nullptr;
+    p.yq = fused ? fused->yq : nullptr;
+    p.ysf = fused ? fused->ysf : nullptr;
+    p.amax_y = fused ? fused->amax_y : nullptr;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.n_sf_blocks = (N + 127) / 128;
+    if (p.amax_y != nullptr) {
+        cudaError_t e = cudaMemsetAsync(p.amax_y, 0, sizeof(float), stream);
+        if (e != cudaSuccess) return NVFP4_ERR_LAUNCH;
+    }
+    return from_cuda(nvfp4::launch_gemm(ta, tb, p, tile_n, sms, stream));
+}
+
+nvfp4_status nvfp4_linear_host(const void *x_host_bf16, int64_t M, int64_t K, const uint8_t *wq,
+                               const uint8_t *wsf, const float *w_s_dec, int64_t N,
+                               void *y_host_bf16, const nvfp4_linear_workspace *ws,
+                               nvfp4_stream_t stream) {
+    if (x_host_bf16 == nullptr || y_host_bf16 == nullptr || ws == nullptr || ws->x == nullptr ||
+        ws->xq == nullptr || ws->xsf == nullptr || ws->amax == nullptr || ws->s_dec == nullptr ||
+        ws->y == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (M < 1 || K < 64 || K % 64 != 0 || N < 8 || N % 8 != 0) return NVFP4_ERR_INVALID_ARG;
+    int sms = 0;
+    nvfp4_status st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    const size_t xbytes = static_cast<size_t>(M) * static_cast<size_t>(K) * 2;
+    const size_t ybytes = static_cast<size_t>(M) * static_cast<size_t>(N) * 2;
+    if (cudaMemcpyAsync(ws->x, x_host_bf16, xbytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+        return NVFP4_ERR_LAUNCH;
+    st = nvfp4_tensor_amax(ws->x, M * K, ws->amax, stream);
+    if (st != NVFP4_OK) return st;
+    st = nvfp4_quantize(ws->x, M, K, ws->amax, ws->xq, ws->xsf, ws->s_dec, stream);
+    if (st != NVFP4_OK) return st;
+    st = nvfp4_gemm(ws->xq, ws->xsf, ws->s_dec, wq, wsf, w_s_dec, M, N, K, ws->y, nullptr, stream);
+    if (st != NVFP4_OK) return st;
+    if (cudaMemcpyAsync(y_host_bf16, ws->y, ybytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return NVFP4_ERR_LAUNCH;
+    return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_device_error(int *code_out, int *detail_out) {
+    if (code_out == nullptr) return NVFP4_ERR_INVALID_ARG;
+    int sms = 0;
+    nvfp4_status st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    int code = 0, detail = 0;
+    if (nvfp4::read_and_clear_device_error(&code, &detail) != cudaSuccess) return NVFP4_ERR_LAUNCH;
+    *code_out = code;
+    if (detail_out != nullptr) *detail_out = detail;
+    return NVFP4_OK;
+}
+
+}  // extern "C"

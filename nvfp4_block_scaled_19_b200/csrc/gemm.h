@@ -1,0 +1,38 @@
+// Host/device interface of the block-scaled FP4 GEMM kernel.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace nvfp4 {
+
+struct GemmParams {
+    const uint8_t *asf;     // A scales, tiled layout, pad128(M) x K/16
+    const uint8_t *bsf;     // B scales, tiled layout, pad128(N) x K/16
+    const float *a_s_dec;   // 1 fp32
+    const float *b_s_dec;   // 1 fp32
+    uint8_t *y;             // bf16 [M,N] or null
+    const float *s_enc_y;   // fused quantize: 1 fp32
+    uint8_t *yq;            // fused quantize: packed [M, N/2] or null (= no fusion)
+    uint8_t *ysf;           // fused quantize: tiled scales
+    float *amax_y;          // fused quantize: 1 fp32 (pre-zeroed) or null
+    int64_t M, N, K;
+    int64_t n_sf_blocks;    // ceil(N / 128): 128-row blocks present in bsf
+};
+
+// Tile width (128 or 256) used for a problem.
+int gemm_tile_n(int64_t M, int64_t N);
+
+cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
+                        int tile_n, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_amax(const void *x, int64_t numel, float *amax, int num_sms,
+                        cudaStream_t stream);
+
+cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, const float *scale_in,
+                            bool dynamic, uint8_t *q, uint8_t *sf, float *s_dec_out, int num_sms,
+                            cudaStream_t stream);
+
+}  // namespace nvfp4

@@ -1,0 +1,107 @@
+// NVFP4 two-level microblock quantization arithmetic on the device: the FP32
+// per-tensor scale and the per-16-element E4M3 block scale ("英伟达B200狂飙
+// 10.2倍！AI绘图告别龟速！", section "NVFP4量化：在精度与速度之间寻得最佳平衡"),
+// with E2M1 elements.  Every fp32 step is one IEEE round-to-nearest-even
+// operation (__fdiv_rn / __fmul_rn), in a fixed order, so the codes are
+// reproducible bit for bit:
+//   S_enc = 2688 / amax (1 if amax == 0, FLT_MAX if not finite)
+//   s     = (a_b / 6) * S_enc ;  sf = E4M3_rn_satfinite(s)
+//   inv   = sf == 0 ? 0 : min(S_enc / sf, FLT_MAX)
+//   q     = E2M1_rn_satfinite(x * inv), sign kept
+// Conversions use the sm_100 cvt.rn.satfinite instructions.
+#pragma once
+
+#include <cfloat>
+#include <cstdint>
+
+namespace nvfp4 {
+
+__device__ __forceinline__ float tensor_encode_scale(float amax) {
+    if (amax == 0.0f) return 1.0f;
+    float s = __fdiv_rn(2688.0f, amax);
+    if (!isfinite(s)) s = FLT_MAX;
+    return s;
+}
+
+// E4M3 code (low byte) of a non-negative fp32 value, round-to-nearest-even,
+// saturating to 448.
+__device__ __forceinline__ uint32_t e4m3_encode(float s) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 h;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 h, %1, %2;\n\t"
+        "cvt.u32.u16 %0, h;\n\t}\n"
+        : "=r"(r)
+        : "f"(0.0f), "f"(s));
+    return r & 0xFFu;
+}
+
+// Value of an unsigned E4M3 code (bias 7; exponent field 0 = subnormal).
+__device__ __forceinline__ float e4m3_decode(uint32_t c) {
+    const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+    return e ? __uint_as_float(((e + 120u) << 23) | (m << 20))
+             : __fmul_rn(static_cast<float>(m), 0.001953125f /* 2^-9 */);
+}
+
+struct BlockScale {
+    uint32_t sf;  // E4M3 code
+    float inv;    // multiplier taking x to E2M1 code space
+};
+
+__device__ __forceinline__ BlockScale block_scale(float a_b, float s_enc) {
+    const float s = __fmul_rn(__fdiv_rn(a_b, 6.0f), s_enc);
+    BlockScale b;
+    b.sf = e4m3_encode(s);
+    const float sfv = e4m3_decode(b.sf);
+    float inv = 0.0f;
+    if (sfv != 0.0f) {
+        inv = __fdiv_rn(s_enc, sfv);
+        if (!isfinite(inv)) inv = FLT_MAX;
+    }
+    b.inv = inv;
+    return b;
+}
+
+// Packs 8 fp32 values (already multiplied by inv) into 8 E2M1 codes, element
+// 2j in the low nibble of byte j.  cvt...e2m1x2 puts its first source
+// operand in the upper nibble.
+__device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v3, float v4,
+                                           float v5, float v6, float v7) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}\n"
+        : "=r"(r)
+        : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+    return r;
+}
+
+// |x| maximum of the 8 bf16 values in a 16-byte word, as bf16 bits (the
+// magnitude order of non-NaN bf16 equals the unsigned order of bits&0x7FFF).
+__device__ __forceinline__ uint32_t absmax_bf16x8(uint4 v) {
+    uint32_t m = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+    return max(m & 0xFFFFu, m >> 16);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// E2M1 codes of 8 bf16 values times inv.
+__device__ __forceinline__ uint32_t quantize_bf16x8(uint4 v, float inv) {
+    return e2m1x8(__fmul_rn(bf16_lo(v.x), inv), __fmul_rn(bf16_hi(v.x), inv),
+                  __fmul_rn(bf16_lo(v.y), inv), __fmul_rn(bf16_hi(v.y), inv),
+                  __fmul_rn(bf16_lo(v.z), inv), __fmul_rn(bf16_hi(v.z), inv),
+                  __fmul_rn(bf16_lo(v.w), inv), __fmul_rn(bf16_hi(v.w), inv));
+}
+
+// Byte offset of the block scale (row r, block c) in the 128x4-tiled layout
+// whose rows hold kb4 = ceil(kb/4) tiles.
+__device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t kb4) {
+    return ((r >> 7) * kb4 + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,112 @@
+"""GPU parity: amax and NVFP4 quantization (bit-exact against the oracle)."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_common import (assert_quant_equal, gpu_quantize_dynamic, oracle_quantize_dynamic,
+                        require_cuda)
+from workloads import WORKLOADS, bf16_bits, draw_x, layer_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    return require_cuda()
+
+
+@pytest.mark.parametrize("numel", [0, 1, 7, 8, 9, 1000, 4096 * 3 + 5, 1 << 22, (1 << 24) + 3])
+def test_amax(nv, orc, numel):
+    g = torch.Generator().manual_seed(numel)
+    x = (torch.randn(max(numel, 1), generator=g) * 3).to(torch.bfloat16)[:numel]
+    if numel > 5:
+        x[numel // 3] = -17.5   # the max sits at a negative value
+    xd = x.cuda()
+    amax = nv.tensor_amax(xd)
+    torch.cuda.synchronize()
+    want = orc.tensor_amax(bf16_bits(x)) if numel else np.float32(0)
+    assert np.float32(amax.item()) == want
+
+
+SMALL_SHAPES = [(1, 16), (3, 48), (127, 80), (128, 64), (130, 272), (257, 512), (64, 3072),
+                (1000, 16), (5, 4096)]
+
+
+@pytest.mark.parametrize("rows,cols", SMALL_SHAPES)
+def test_quantize_small_shapes(nv, rows, cols):
+    x = draw_x("normal_outliers", rows, cols, seed=rows * 7 + cols, index=0)
+    assert_quant_equal(gpu_quantize_dynamic(nv, x), oracle_quantize_dynamic(x), f"{rows}x{cols}")
+
+
+def _edge_tensor(kind, rows=130, cols=80):
+    g = torch.Generator().manual_seed(11)
+    if kind == "zeros":
+        return torch.zeros(rows, cols, dtype=torch.bfloat16)
+    if kind == "negative_zeros":
+        return torch.full((rows, cols), -0.0, dtype=torch.bfloat16)
+    if kind == "mixed_zero_blocks":
+        x = torch.randn(rows, cols, generator=g)
+        x[:, 16:32] = 0.0
+        x[::3, 48:64] = -0.0
+        return x.to(torch.bfloat16)
+    if kind == "bf16_subnormals":
+        x = torch.randn(rows, cols, generator=g) * 2.0 ** -128
+        return x.to(torch.bfloat16)
+    if kind == "subnormals_with_zeros":
+        x = torch.randn(rows, cols, generator=g) * 2.0 ** -130
+        x[:, ::5] = 0.0
+        return x.to(torch.bfloat16)
+    if kind == "huge":
+        x = torch.randn(rows, cols, generator=g) * 1e37
+        x[0, 0] = 3.0e38
+        return x.to(torch.bfloat16)
+    if kind == "underflow_blocks":
+        x = torch.randn(rows, cols, generator=g) * 1e-6
+        x[:, :16] = torch.randn(rows, 16, generator=g) * 1e4
+        return x.to(torch.bfloat16)
+    if kind == "one_hot":
+        x = torch.zeros(rows, cols)
+        x[torch.arange(rows), torch.arange(rows) % cols] = torch.linspace(-5, 5, rows)
+        return x.to(torch.bfloat16)
+    if kind == "ties":
+        # Values that land exactly on E2M1 midpoints after scaling by inv=1:
+        # blocks with amax 6 and S_enc = 2688/6 give sf = 448 and inv = 1.
+        mids = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0])
+        x = mids.repeat(rows, cols // 8)
+        x = x * torch.where(torch.rand(rows, cols, generator=g) < 0.5, -1.0, 1.0)
+        return x.to(torch.bfloat16)
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("kind", ["zeros", "negative_zeros", "mixed_zero_blocks",
+                                  "bf16_subnormals", "subnormals_with_zeros", "huge",
+                                  "underflow_blocks", "one_hot", "ties"])
+def test_quantize_edge_cases(nv, kind):
+    x = _edge_tensor(kind)
+    assert_quant_equal(gpu_quantize_dynamic(nv, x), oracle_quantize_dynamic(x), kind)
+
+
+def test_quantize_static_scale(nv, orc):
+    g = torch.Generator().manual_seed(3)
+    x = (torch.randn(200, 96, generator=g) * 4).to(torch.bfloat16)
+    for s in (1.0, 0.37, 448.0, 2.0 ** -20):
+        s_enc = torch.tensor([s], dtype=torch.float32, device="cuda")
+        t = nv.quantize_with_scale(x.cuda(), s_enc)
+        torch.cuda.synchronize()
+        oq, osf = orc.quantize(bf16_bits(x), 200, 96, np.float32(s))
+        assert np.array_equal(t.q.cpu().numpy(), oq)
+        assert np.array_equal(t.sf.cpu().numpy(), osf)
+        assert np.float32(t.s_dec.item()) == orc.decode_scale(np.float32(s))
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_quantize_workloads_full_size(nv, name):
+    """Activations and weights of every workload, at full size, bit-exact."""
+    w = WORKLOADS[name]
+    for li in range(len(w.layers)):
+        x, wt = layer_inputs(w, li)
+        assert_quant_equal(gpu_quantize_dynamic(nv, x), oracle_quantize_dynamic(x),
+                           f"{name}/{w.layers[li].name}/X")
+        assert_quant_equal(gpu_quantize_dynamic(nv, wt), oracle_quantize_dynamic(wt),
+                           f"{name}/{w.layers[li].name}/W")
+        del x, wt
