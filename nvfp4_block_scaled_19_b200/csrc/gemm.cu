@@ -4,8 +4,8 @@
 // optionally followed by the next layer's NVFP4 quantization of Y in the
 // epilogue.  This is the NVFP4 linear layer of the FLUX DiT pages ("英伟达
 // B200狂飙10.2倍！AI绘图告别龟速！", section "NVFP4量化"; the NVFP4 GEMM kernels
-// compared in "NVIDIA shows how TensorRT-LLM VisualGen speeds up FLUX 3 Image
-// Klein on Blackwell", optimisation section), written here from scratch.
+// compared in "NVIDIA介绍用TensorRT LLM VisualGen加速Blackwell上的FLUX 3 Image
+// Klein", paragraph on the tested optimisations), written here from scratch.
 //
 // Design (persistent, warp-specialised, one CTA per SM, 128 x BN tiles):
 //   warp 0        TMA producer: per k-stage of 256 elements, a 2-D TMA load of

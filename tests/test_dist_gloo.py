@@ -1,0 +1,62 @@
+"""The multi-process (N > 1) bench plumbing on CPU with gloo, world size 2:
+max-over-ranks timing, whole-job aggregation of replicas, and rank-0-only
+output of the reference arm."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import bench
+    dist = bench.init_dist(world, "gloo")
+    dev = torch.device("cpu")
+    t = bench.max_over_ranks(1.5 + rank, dist, dev)       # rank 1 is the slow one
+    bench.barrier(dist, dev)
+    v = bench.aggregate(per_rank_units=10.0, world=world, max_seconds=t)
+    out[rank] = (t, v, bench.dist_env())
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_two_rank_timing_and_aggregation():
+    world = 2
+    port = _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+    for r in range(world):
+        t, v, env = out[r]
+        assert t == 2.5                 # the max over ranks, on every rank
+        assert v == pytest.approx(10.0 * 2 / 2.5)
+        assert env == (r, world, r)
+
+
+def test_single_process_defaults(monkeypatch):
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    import bench
+    assert bench.dist_env() == (0, 1, 0)
+    assert bench.init_dist(1, "gloo") is None
+    assert bench.max_over_ranks(3.0, None, torch.device("cpu")) == 3.0
+    assert bench.aggregate(5.0, 1, 2.0) == 2.5
+
+
+def test_reference_arm_only_rank0_prints(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    import bench
+    assert bench.reference_arm(bench.argparse.Namespace(
+        workload="tiny_linear", warmup=1, steps=1, cpu_rows=16)) is None

@@ -5,14 +5,15 @@ of FLUX diffusion-transformer linear layers. It holds none of the NVFP4
 arithmetic (no amax, scales, rounding or packing), so both the CPU oracle and
 the CUDA path can take their inputs from it without sharing method code.
 
-Sources for the shapes: the FLUX pages describe a DiT with joint attention
-over image and text tokens ("NVIDIA shows how TensorRT-LLM VisualGen speeds up
-FLUX 3 Image Klein on Blackwell", the time-breakdown section; "Scaling NVFP4
-Inference for FLUX.2 on NVIDIA Blackwell Data Center GPUs", Overview). The
-token counts (4096 image + 512 text tokens at 1024^2, 16384 + 512 at 2048^2,
-doubled for a classifier-free-guidance batch of 2), hidden size 3072 and FFN
-width 12288 are this library's synthetic stand-ins; no trained weights,
-prompts or images are used.
+Sources for the shapes: the FLUX pages describe a DiT that mixes text and
+image tokens with joint attention ("NVIDIA показала, как сократить генерацию
+FLUX 3 Image Klein с 22 до 6 секунд", section "Как устроена FLUX 3 Image
+Klein") and time its 2048x2048 runs with classifier-free guidance ("NVIDIA
+介绍用TensorRT LLM VisualGen加速Blackwell上的FLUX 3 Image Klein", paragraph on
+the time breakdown).  The token counts (4096 image + 512 text tokens at
+1024^2, 16384 + 512 at 2048^2, doubled for a guidance batch of 2), hidden
+size 3072 and FFN width 12288 are this library's synthetic stand-ins; no
+trained weights, prompts or images are used.
 
 Every tensor is drawn from its own torch CPU generator seeded from the
 workload seed and the tensor's index, as float32, transformed, then rounded
