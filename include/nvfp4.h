@@ -120,6 +120,26 @@ nvfp4_status nvfp4_quantize_with_scale(const void *x_bf16, int64_t rows, int64_t
                                        uint8_t *sf_out, float *s_dec_out,
                                        nvfp4_stream_t stream);
 
+/* Bytes of device workspace needed by nvfp4_quantize_dynamic (32). */
+size_t nvfp4_quantize_dynamic_workspace_bytes(void);
+
+/* Dynamic NVFP4 quantization in one launch: the per-tensor amax, S_enc and
+ * the per-16 block quantization of nvfp4_tensor_amax + nvfp4_quantize
+ * (nmedialink page above, NVFP4 section: dynamic per-tensor and per-block
+ * scales), with identical results.  A cooperative kernel reduces the amax,
+ * crosses one grid barrier and quantizes, reading the tensor from L2 the
+ * second time where it fits.
+ *   x_bf16, rows, cols, q_out, sf_out, s_dec_out  as for nvfp4_quantize
+ *   amax_out   device, 1 fp32, written with max|x| (NULL = not written)
+ *   workspace  device, nvfp4_quantize_dynamic_workspace_bytes() bytes,
+ *              16-byte aligned, zero-filled once by the caller before its
+ *              first use and then reused unchanged; calls that share a
+ *              workspace must be ordered (same stream, or synchronised).
+ *              After an NVFP4_ERR_TIMEOUT it must be zero-filled again. */
+nvfp4_status nvfp4_quantize_dynamic(const void *x_bf16, int64_t rows, int64_t cols,
+                                    uint8_t *q_out, uint8_t *sf_out, float *s_dec_out,
+                                    float *amax_out, void *workspace, nvfp4_stream_t stream);
+
 /* Block-scaled FP4 GEMM on tcgen05 tensor cores, Y = X . W^T (the NVFP4
  * linear layer whose weights are quantized once, "quantize_weights=True",
  * nmedialink page above, NVFP4 section).
@@ -137,7 +157,9 @@ nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_
 
 /* Device buffers for nvfp4_linear_host (all caller-owned device memory):
  *   x      [M,K] bf16      xq  M*K/2 bytes      xsf  nvfp4_sf_bytes(M,K)
- *   amax   1 fp32          s_dec 1 fp32         y    [M,N] bf16 */
+ *   amax   1 fp32          s_dec 1 fp32         y    [M,N] bf16
+ *   dyn_ws workspace of nvfp4_quantize_dynamic (zero-filled once), or NULL
+ *          to quantize with nvfp4_tensor_amax + nvfp4_quantize */
 typedef struct {
     void *x;
     uint8_t *xq;
@@ -145,6 +167,7 @@ typedef struct {
     float *amax;
     float *s_dec;
     void *y;
+    void *dyn_ws;
 } nvfp4_linear_workspace;
 
 /* One NVFP4 linear layer from host memory: copies X host->device, runs

@@ -40,7 +40,8 @@ class FusedOut(ctypes.Structure):
 
 class LinearWorkspace(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("xq", ctypes.c_void_p), ("xsf", ctypes.c_void_p),
-                ("amax", ctypes.c_void_p), ("s_dec", ctypes.c_void_p), ("y", ctypes.c_void_p)]
+                ("amax", ctypes.c_void_p), ("s_dec", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("dyn_ws", ctypes.c_void_p)]
 
 
 _lib = None
@@ -67,6 +68,10 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_quantize.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
         L.nvfp4_quantize_with_scale.restype = st
         L.nvfp4_quantize_with_scale.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
+        L.nvfp4_quantize_dynamic_workspace_bytes.restype = ctypes.c_size_t
+        L.nvfp4_quantize_dynamic_workspace_bytes.argtypes = []
+        L.nvfp4_quantize_dynamic.restype = st
+        L.nvfp4_quantize_dynamic.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp, vp]
         L.nvfp4_gemm.restype = st
         L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp,
                                  ctypes.POINTER(FusedOut), vp]
@@ -157,11 +162,33 @@ def quantize_with_scale(x: torch.Tensor, s_enc: torch.Tensor, out: NVFP4Tensor |
     return out
 
 
+_dyn_workspaces: dict = {}
+
+
+def dynamic_workspace(device=None) -> torch.Tensor:
+    """A zero-filled workspace for nvfp4_quantize_dynamic (one per device,
+    shared by calls on one stream; give concurrent streams their own)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    ws = _dyn_workspaces.get(dev)
+    if ws is None:
+        n = int(lib().nvfp4_quantize_dynamic_workspace_bytes())
+        ws = torch.zeros((n + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+        _dyn_workspaces[dev] = ws
+    return ws
+
+
 def quantize_dynamic(x: torch.Tensor, out: NVFP4Tensor | None = None,
-                     amax: torch.Tensor | None = None, stream=None) -> NVFP4Tensor:
-    """amax then quantize: the per-call activation path."""
-    amax = tensor_amax(x, amax, stream)
-    return quantize(x, amax, out, stream)
+                     amax: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                     stream=None) -> NVFP4Tensor:
+    """Per-call activation path in one launch: amax, S_enc, block quantize."""
+    _require(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    out = empty_nvfp4(rows, cols, x.device) if out is None else out
+    ws = dynamic_workspace(x.device) if workspace is None else workspace
+    _check("nvfp4_quantize_dynamic", lib().nvfp4_quantize_dynamic(
+        x.data_ptr(), rows, cols, out.q.data_ptr(), out.sf.data_ptr(), out.s_dec.data_ptr(),
+        _ptr(amax), ws.data_ptr(), _stream(stream)))
+    return out
 
 
 @dataclass
@@ -221,7 +248,8 @@ class NVFP4Linear:
         """Host bf16 X -> host bf16 Y through nvfp4_linear_host (copies included)."""
         M = x_host.shape[0]
         w = LinearWorkspace(ws["x"].data_ptr(), ws["xq"].data_ptr(), ws["xsf"].data_ptr(),
-                            ws["amax"].data_ptr(), ws["s_dec"].data_ptr(), ws["y"].data_ptr())
+                            ws["amax"].data_ptr(), ws["s_dec"].data_ptr(), ws["y"].data_ptr(),
+                            dynamic_workspace(ws["x"].device).data_ptr())
         _check("nvfp4_linear_host", lib().nvfp4_linear_host(
             x_host.data_ptr(), M, self.K, self.w.q.data_ptr(), self.w.sf.data_ptr(),
             self.w.s_dec.data_ptr(), self.N, y_host.data_ptr(), ctypes.byref(w),

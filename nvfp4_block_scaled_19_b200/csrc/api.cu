@@ -157,6 +157,31 @@ nvfp4_status nvfp4_quantize_with_scale(const void *x_bf16, int64_t rows, int64_t
     return quantize_impl(x_bf16, rows, cols, s_enc_dev, false, q_out, sf_out, s_dec_out, stream);
 }
 
+size_t nvfp4_quantize_dynamic_workspace_bytes(void) { return sizeof(nvfp4::DynWorkspace); }
+
+nvfp4_status nvfp4_quantize_dynamic(const void *x_bf16, int64_t rows, int64_t cols, uint8_t *q_out,
+                                    uint8_t *sf_out, float *s_dec_out, float *amax_out,
+                                    void *workspace, nvfp4_stream_t stream) {
+    nvfp4_status st = check_quantize_args(x_bf16, rows, cols, workspace, q_out, sf_out);
+    if (st != NVFP4_OK) return st;
+    if (!aligned16(workspace)) return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    nvfp4::DynWorkspace *ws = static_cast<nvfp4::DynWorkspace *>(workspace);
+    cudaError_t e = nvfp4::launch_quantize_dynamic(x_bf16, rows, cols, q_out, sf_out, s_dec_out,
+                                                   amax_out, ws, sms, stream);
+    if (e == cudaErrorNotSupported) {
+        cudaGetLastError();
+        float *amax = amax_out != nullptr ? amax_out : &ws->fallback_amax;
+        e = nvfp4::launch_amax(x_bf16, rows * cols, amax, sms, stream);
+        if (e == cudaSuccess)
+            e = nvfp4::launch_quantize(x_bf16, rows, cols, amax, true, q_out, sf_out, s_dec_out,
+                                       sms, stream);
+    }
+    return from_cuda(e);
+}
+
 nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_dec,
                         const uint8_t *bq, const uint8_t *bsf, const float *b_s_dec, int64_t M,
                         int64_t N, int64_t K, void *y_bf16, const nvfp4_fused_out *fused,
@@ -226,9 +251,14 @@ nvfp4_status nvfp4_linear_host(const void *x_host_bf16, int64_t M, int64_t K, co
     const size_t ybytes = static_cast<size_t>(M) * static_cast<size_t>(N) * 2;
     if (cudaMemcpyAsync(ws->x, x_host_bf16, xbytes, cudaMemcpyHostToDevice, stream) != cudaSuccess)
         return NVFP4_ERR_LAUNCH;
-    st = nvfp4_tensor_amax(ws->x, M * K, ws->amax, stream);
-    if (st != NVFP4_OK) return st;
-    st = nvfp4_quantize(ws->x, M, K, ws->amax, ws->xq, ws->xsf, ws->s_dec, stream);
+    if (ws->dyn_ws != nullptr) {
+        st = nvfp4_quantize_dynamic(ws->x, M, K, ws->xq, ws->xsf, ws->s_dec, ws->amax, ws->dyn_ws,
+                                    stream);
+    } else {
+        st = nvfp4_tensor_amax(ws->x, M * K, ws->amax, stream);
+        if (st == NVFP4_OK)
+            st = nvfp4_quantize(ws->x, M, K, ws->amax, ws->xq, ws->xsf, ws->s_dec, stream);
+    }
     if (st != NVFP4_OK) return st;
     st = nvfp4_gemm(ws->xq, ws->xsf, ws->s_dec, wq, wsf, w_s_dec, M, N, K, ws->y, nullptr, stream);
     if (st != NVFP4_OK) return st;

@@ -46,14 +46,25 @@ namespace nvfp4 {
 cudaError_t read_and_clear_device_error(int *code, int *detail) {
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return e;
-    e = cudaMemcpyFromSymbol(code, g_error_code, sizeof(int));
+    int v[2] = {0, 0};
+    e = cudaMemcpyFromSymbol(v, g_error, sizeof(v));
     if (e != cudaSuccess) return e;
-    e = cudaMemcpyFromSymbol(detail, g_error_detail, sizeof(int));
-    if (e != cudaSuccess) return e;
-    const int zero = 0;
-    e = cudaMemcpyToSymbol(g_error_code, &zero, sizeof(int));
-    if (e != cudaSuccess) return e;
-    return cudaMemcpyToSymbol(g_error_detail, &zero, sizeof(int));
+    *code = v[0];
+    *detail = v[1];
+    const int zero[2] = {0, 0};
+    return cudaMemcpyToSymbol(g_error, zero, sizeof(zero));
+}
+
+int *device_error_word() {
+    static int *addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (addr[dev] == nullptr) {
+        void *a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_error) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int *>(a);
+    }
+    return addr[dev];
 }
 
 constexpr int kBM = 128;

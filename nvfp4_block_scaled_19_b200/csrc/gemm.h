@@ -22,6 +22,10 @@ struct GemmParams {
     int64_t n_sf_blocks;    // ceil(N / 128): 128-row blocks present in bsf
 };
 
+// Device address of the library's error word (int[2]: code, tag) on the
+// current device, for kernels outside the GEMM translation unit.
+int *device_error_word();
+
 // Tile width (128 or 256) used for a problem.
 int gemm_tile_n(int64_t M, int64_t N);
 
@@ -34,5 +38,21 @@ cudaError_t launch_amax(const void *x, int64_t numel, float *amax, int num_sms,
 cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, const float *scale_in,
                             bool dynamic, uint8_t *q, uint8_t *sf, float *s_dec_out, int num_sms,
                             cudaStream_t stream);
+
+// Workspace of the single-launch dynamic quantization (zero-initialised once
+// by the caller; calls that share one must be stream-ordered).
+struct DynWorkspace {
+    unsigned count;         // CTAs arrived at the grid barrier (back to 0 after it)
+    unsigned gen;           // barrier generation, +1 per launch
+    unsigned amax_bits[2];  // amax of launch g in [g & 1]; the other is cleared
+    float fallback_amax;    // used when rows are too wide for one cooperative grid
+    unsigned pad[3];
+};
+
+// Returns cudaErrorNotSupported when the rows are too wide for one
+// cooperative grid (then use launch_amax + launch_quantize).
+cudaError_t launch_quantize_dynamic(const void *x, int64_t rows, int64_t cols, uint8_t *q,
+                                    uint8_t *sf, float *s_dec_out, float *amax_out,
+                                    DynWorkspace *ws, int num_sms, cudaStream_t stream);
 
 }  // namespace nvfp4

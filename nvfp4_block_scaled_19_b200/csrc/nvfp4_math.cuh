@@ -87,6 +87,43 @@ __device__ __forceinline__ uint32_t absmax_bf16x8(uint4 v) {
     return max(m & 0xFFFFu, m >> 16);
 }
 
+// 16 bf16 values (32 bytes) held as 8 words.
+struct BF16x16 {
+    uint32_t w[8];
+};
+
+__device__ __forceinline__ BF16x16 ldg_stream_32B(const void *p) {
+    BF16x16 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]),
+                   "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
+                 : "l"(p));
+    return v;
+}
+
+// 32 bytes at p: one 256-bit load when p is 32-byte aligned, else two
+// 128-bit loads (the ABI only guarantees 16-byte alignment).
+__device__ __forceinline__ BF16x16 ldg_32B(const uint8_t *p, bool aligned32) {
+    if (aligned32) return ldg_stream_32B(p);
+    BF16x16 v;
+    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
+    const uint4 b = __ldg(reinterpret_cast<const uint4 *>(p + 16));
+    v.w[0] = a.x; v.w[1] = a.y; v.w[2] = a.z; v.w[3] = a.w;
+    v.w[4] = b.x; v.w[5] = b.y; v.w[6] = b.z; v.w[7] = b.w;
+    return v;
+}
+
+__device__ __forceinline__ uint32_t absmax_bf16x16(const BF16x16 &v) {
+    uint32_t m = __vmaxu2(v.w[0] & 0x7FFF7FFFu, v.w[1] & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.w[2] & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.w[3] & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.w[4] & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.w[5] & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.w[6] & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v.w[7] & 0x7FFF7FFFu);
+    return max(m & 0xFFFFu, m >> 16);
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 

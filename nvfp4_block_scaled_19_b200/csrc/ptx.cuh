@@ -12,8 +12,9 @@ namespace nvfp4 {
 // Device-side error word (NVFP4_ERR_TIMEOUT when a bounded wait gives up)
 // and a tag saying which wait it was.  Defined here because exactly one
 // translation unit (gemm.cu, the only kernel with waits) includes this file.
-__device__ int g_error_code = 0;
-__device__ int g_error_detail = 0;
+// g_error[0] = code, g_error[1] = detail.  Kernels in other translation units
+// receive its device address (device_error_word()) as a parameter.
+__device__ int g_error[2] = {0, 0};
 
 // A wait gives up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
@@ -29,7 +30,7 @@ __device__ __forceinline__ uint64_t globaltimer() {
 }
 
 __device__ __forceinline__ void record_timeout(int tag) {
-    if (atomicCAS(&g_error_code, 0, 5) == 0) g_error_detail = tag;
+    if (atomicCAS(&g_error[0], 0, 5) == 0) g_error[1] = tag;
 }
 
 // ------------------------------------------------------------------ mbarrier

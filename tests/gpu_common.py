@@ -17,12 +17,20 @@ def require_cuda():
     return nv
 
 
-def gpu_quantize_dynamic(nv, x_cpu):
-    """amax + dynamic quantize on the GPU -> numpy (q, sf, s_dec, amax)."""
+def gpu_quantize_dynamic(nv, x_cpu, path="fused"):
+    """Dynamic quantize on the GPU -> numpy (q, sf, s_dec, amax).
+    path "two_kernel": nvfp4_tensor_amax + nvfp4_quantize;
+    path "fused": nvfp4_quantize_dynamic (one cooperative launch)."""
     x = x_cpu.cuda()
-    amax = nv.tensor_amax(x)
-    t = nv.quantize(x, amax)
+    if path == "two_kernel":
+        amax = nv.tensor_amax(x)
+        t = nv.quantize(x, amax)
+    else:
+        amax = torch.full((1,), -1.0, device="cuda")
+        t = nv.quantize_dynamic(x, amax=amax)
     torch.cuda.synchronize()
+    code, tag = nv.device_error()
+    assert code == 0, f"device wait timed out (tag {tag})"
     return (t.q.cpu().numpy(), t.sf.cpu().numpy(), np.float32(t.s_dec.item()),
             np.float32(amax.item()))
 

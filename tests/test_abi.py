@@ -31,7 +31,8 @@ def test_header_declares_the_boundary():
     names = _declared_functions()
     for n in ("nvfp4_tensor_amax", "nvfp4_quantize", "nvfp4_quantize_with_scale", "nvfp4_gemm",
               "nvfp4_packed_bytes", "nvfp4_sf_bytes", "nvfp4_status_string",
-              "nvfp4_linear_host", "nvfp4_device_error"):
+              "nvfp4_linear_host", "nvfp4_device_error", "nvfp4_quantize_dynamic",
+              "nvfp4_quantize_dynamic_workspace_bytes"):
         assert n in names
 
 
@@ -86,6 +87,11 @@ def test_invalid_arguments_rejected_first(L):
     ok = nv.FusedOut(p, p, p, None)
     assert g(p, p, p, p, p, p, 128, 120, 128, p, ctypes.byref(ok), None) == 1  # N % 16
     assert L.nvfp4_device_error(None, None) == 1
+    qd = L.nvfp4_quantize_dynamic
+    assert qd(p, 4, 24, p, p, None, None, p, None) == 1         # cols % 16
+    assert qd(p, 4, 32, p, p, None, None, None, None) == 1      # no workspace
+    assert qd(p, 4, 32, p, p, None, None, p + 4, None) == 2     # misaligned workspace
+    assert L.nvfp4_quantize_dynamic_workspace_bytes() == 32
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device answer")

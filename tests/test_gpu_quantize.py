@@ -32,10 +32,15 @@ SMALL_SHAPES = [(1, 16), (3, 48), (127, 80), (128, 64), (130, 272), (257, 512), 
                 (1000, 16), (5, 4096)]
 
 
+PATHS = ["two_kernel", "fused"]
+
+
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("rows,cols", SMALL_SHAPES)
-def test_quantize_small_shapes(nv, rows, cols):
+def test_quantize_small_shapes(nv, rows, cols, path):
     x = draw_x("normal_outliers", rows, cols, seed=rows * 7 + cols, index=0)
-    assert_quant_equal(gpu_quantize_dynamic(nv, x), oracle_quantize_dynamic(x), f"{rows}x{cols}")
+    assert_quant_equal(gpu_quantize_dynamic(nv, x, path), oracle_quantize_dynamic(x),
+                       f"{rows}x{cols}/{path}")
 
 
 def _edge_tensor(kind, rows=130, cols=80):
@@ -78,12 +83,27 @@ def _edge_tensor(kind, rows=130, cols=80):
     raise ValueError(kind)
 
 
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("kind", ["zeros", "negative_zeros", "mixed_zero_blocks",
                                   "bf16_subnormals", "subnormals_with_zeros", "huge",
                                   "underflow_blocks", "one_hot", "ties"])
-def test_quantize_edge_cases(nv, kind):
+def test_quantize_edge_cases(nv, kind, path):
     x = _edge_tensor(kind)
-    assert_quant_equal(gpu_quantize_dynamic(nv, x), oracle_quantize_dynamic(x), kind)
+    assert_quant_equal(gpu_quantize_dynamic(nv, x, path), oracle_quantize_dynamic(x),
+                       f"{kind}/{path}")
+
+
+def test_quantize_dynamic_back_to_back(nv):
+    """Consecutive single-launch quantizations of different shapes (different
+    cooperative grid sizes) share one workspace: every result must be exact,
+    so the grid barrier and the per-launch amax words reset correctly."""
+    shapes = [(257, 512), (64, 3072), (1, 16), (4608, 3072), (130, 272), (1000, 12288),
+              (3, 48), (257, 512)]
+    for i, (rows, cols) in enumerate(shapes):
+        x = draw_x("lognormal_channels", rows, cols, seed=100 + i, index=0)
+        x = (x * (10.0 ** (i % 5 - 2))).to(torch.bfloat16)   # amax changes every call
+        assert_quant_equal(gpu_quantize_dynamic(nv, x, "fused"), oracle_quantize_dynamic(x),
+                           f"call {i} {rows}x{cols}")
 
 
 def test_quantize_static_scale(nv, orc):
@@ -101,12 +121,35 @@ def test_quantize_static_scale(nv, orc):
 
 @pytest.mark.parametrize("name", list(WORKLOADS))
 def test_quantize_workloads_full_size(nv, name):
-    """Activations and weights of every workload, at full size, bit-exact."""
+    """Activations (per-call, single-launch path) and weights (load-time,
+    two-kernel path) of every workload, at full size, bit-exact."""
     w = WORKLOADS[name]
     for li in range(len(w.layers)):
         x, wt = layer_inputs(w, li)
-        assert_quant_equal(gpu_quantize_dynamic(nv, x), oracle_quantize_dynamic(x),
+        assert_quant_equal(gpu_quantize_dynamic(nv, x, "fused"), oracle_quantize_dynamic(x),
                            f"{name}/{w.layers[li].name}/X")
-        assert_quant_equal(gpu_quantize_dynamic(nv, wt), oracle_quantize_dynamic(wt),
-                           f"{name}/{w.layers[li].name}/W")
+        assert_quant_equal(gpu_quantize_dynamic(nv, wt, "two_kernel"),
+                           oracle_quantize_dynamic(wt), f"{name}/{w.layers[li].name}/W")
         del x, wt
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_quantize_input_16_byte_aligned(nv, path):
+    """An input that is 16-byte but not 32-byte aligned (a view 8 elements
+    into a buffer) takes the two-load path and gives the same codes."""
+    rows, cols = 130, 272
+    x = draw_x("normal_outliers", rows, cols, seed=77, index=0)
+    buf = torch.zeros(rows * cols + 16, dtype=torch.bfloat16, device="cuda")
+    view = buf[8:8 + rows * cols].view(rows, cols)
+    assert view.data_ptr() % 32 == 16
+    view.copy_(x.cuda())
+    if path == "two_kernel":
+        amax = nv.tensor_amax(view)
+        t = nv.quantize(view, amax)
+    else:
+        amax = torch.empty(1, device="cuda")
+        t = nv.quantize_dynamic(view, amax=amax)
+    torch.cuda.synchronize()
+    got = (t.q.cpu().numpy(), t.sf.cpu().numpy(), np.float32(t.s_dec.item()),
+           np.float32(amax.item()))
+    assert_quant_equal(got, oracle_quantize_dynamic(x), f"16B-aligned/{path}")
