@@ -140,6 +140,28 @@ nvfp4_status nvfp4_quantize_dynamic(const void *x_bf16, int64_t rows, int64_t co
                                     uint8_t *q_out, uint8_t *sf_out, float *s_dec_out,
                                     float *amax_out, void *workspace, nvfp4_stream_t stream);
 
+/* nvfp4_quantize_dynamic for callers that cannot allocate device memory: an
+ * inference-engine plugin whose execute step may not allocate, a runtime
+ * that owns all device memory through its own arena, or a latency-critical
+ * loop that must avoid cudaMalloc/cudaFree because they can synchronise the
+ * device.  No counterpart on the pages: it is the same computation with the
+ * same results as nvfp4_quantize_dynamic, and allocates nothing.
+ *   x_bf16, rows, cols, q_out, sf_out, s_dec_out, amax_out
+ *              as for nvfp4_quantize_dynamic (the caller still provides every
+ *              input and output)
+ * Scratch: instead of a caller workspace the call uses a 256-byte array
+ * inside the library (every GPU that loads the library holds it until the
+ * process exits).  The call clears the part it needs on `stream` before
+ * using it.  The scratch needed is 32 bytes for any tensor size; a call that
+ * would need more than 256 bytes is refused with NVFP4_ERR_INVALID_ARG.
+ * The first call on a device looks up the array's device address, so make
+ * that first call before any stream capture.  All calls on a device share
+ * the one array: calls that overlap on the GPU (on streams not ordered with
+ * each other) race on it and give wrong results. */
+nvfp4_status nvfp4_quantize_dynamic_noalloc(const void *x_bf16, int64_t rows, int64_t cols,
+                                            uint8_t *q_out, uint8_t *sf_out, float *s_dec_out,
+                                            float *amax_out, nvfp4_stream_t stream);
+
 /* Block-scaled FP4 GEMM on tcgen05 tensor cores, Y = X . W^T (the NVFP4
  * linear layer whose weights are quantized once, "quantize_weights=True",
  * nmedialink page above, NVFP4 section).
