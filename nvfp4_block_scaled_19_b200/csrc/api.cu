@@ -205,13 +205,13 @@ nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_
     nvfp4_status st = current_device(&sms);
     if (st != NVFP4_OK) return st;
 
-    const int tile_n = nvfp4::gemm_tile_n(M, N);
+    const nvfp4::GemmKind kind = nvfp4::gemm_kind(M, N);
     CUtensorMap ta, tb;
     std::memset(&ta, 0, sizeof(ta));
     std::memset(&tb, 0, sizeof(tb));
     if (!encode_operand_map(&ta, aq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M), 128) ||
         !encode_operand_map(&tb, bq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N),
-                            static_cast<uint32_t>(tile_n)))
+                            nvfp4::gemm_b_box_rows(kind)))
         return NVFP4_ERR_LAUNCH;
 
     nvfp4::GemmParams p;
@@ -228,11 +228,12 @@ nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_
     p.N = N;
     p.K = K;
     p.n_sf_blocks = (N + 127) / 128;
+    p.m_sf_blocks = (M + 127) / 128;
     if (p.amax_y != nullptr) {
         cudaError_t e = cudaMemsetAsync(p.amax_y, 0, sizeof(float), stream);
         if (e != cudaSuccess) return NVFP4_ERR_LAUNCH;
     }
-    return from_cuda(nvfp4::launch_gemm(ta, tb, p, tile_n, sms, stream));
+    return from_cuda(nvfp4::launch_gemm(ta, tb, p, kind, sms, stream));
 }
 
 nvfp4_status nvfp4_linear_host(const void *x_host_bf16, int64_t M, int64_t K, const uint8_t *wq,

@@ -38,6 +38,7 @@
 #include <cstdint>
 
 #include "gemm.h"
+#include "gemm_common.cuh"
 #include "nvfp4_math.cuh"
 #include "ptx.cuh"
 
@@ -106,26 +107,6 @@ struct GemmConfig {
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t IDESC = make_idesc_mxf4nvf4(kBM, BN);
 };
-
-struct TileCoord {
-    int m_blk, n_blk;
-};
-
-// Tile t -> (m, n) block, walking groups of kGroupM row-blocks with m fastest
-// inside a group, so concurrently running CTAs share B (weight) tiles and a
-// group's A rows stay in L2.
-constexpr int kGroupM = 8;
-__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n) {
-    const int per_group = kGroupM * tiles_n;
-    const int g = t / per_group;
-    const int first_m = g * kGroupM;
-    const int gsz = min(tiles_m - first_m, kGroupM);
-    const int r = t - g * per_group;
-    TileCoord c;
-    c.m_blk = first_m + r % gsz;
-    c.n_blk = r / gsz;
-    return c;
-}
 
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
@@ -343,7 +324,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sf_full[stage]);
+                if (lane == 0) mbar_arrive_relaxed(&sf_full[stage]);
                 if (++stage == Cfg::STAGES) {
                     stage = 0;
                     phase ^= 1;
@@ -357,10 +338,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int col0 = (e >> 2) * 128;  // this warp's 128 columns of the tile
         const int row_in_tile = quad * 32 + lane;
         const float alpha = __fmul_rn(*p.a_s_dec, *p.b_s_dec);
-        const bool fused = p.yq != nullptr;
-        const float s_enc_y = fused ? *p.s_enc_y : 1.0f;
-        const int64_t nb_y = p.N / 16;
-        const int64_t nb4_y = (nb_y + 3) / 4;
+        const float s_enc_y = p.yq != nullptr ? *p.s_enc_y : 1.0f;
         uint32_t amax_bits = 0;
         int local = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
@@ -371,81 +349,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             tc_fence_after();
             // Drain 128 accumulator columns into 64 packed bf16x2 registers.
             uint32_t pk[64];
-            const uint32_t taddr =
-                tmem_base + acc * Cfg::BN + col0 + ((static_cast<uint32_t>(quad) * 32) << 16);
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(taddr + ch * 32, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const __nv_bfloat162 h =
-                        __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
-                                              __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
-                    pk[16 * ch + i] = *reinterpret_cast<const uint32_t *>(&h);
-                }
-            }
+            drain_128(tmem_base + acc * Cfg::BN + col0 + ((static_cast<uint32_t>(quad) * 32) << 16),
+                      alpha, pk);
             // Accumulator read: hand it back to the MMA warp.
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
-
-            const int64_t m = int64_t(tc.m_blk) * kBM + row_in_tile;
-            const bool row_ok = m < p.M;
-            const int64_t n0 = int64_t(tc.n_blk) * Cfg::BN + col0;
-            if (row_ok && p.y != nullptr) {
-                uint8_t *yrow = p.y + (m * p.N + n0) * 2;
-                if (n0 + 128 <= p.N && (p.N & 15) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 31) == 0) {
-#pragma unroll
-                    for (int g = 0; g < 8; ++g)
-                        stg256(yrow + 32 * g, pk[8 * g], pk[8 * g + 1], pk[8 * g + 2],
-                               pk[8 * g + 3], pk[8 * g + 4], pk[8 * g + 5], pk[8 * g + 6],
-                               pk[8 * g + 7]);
-                } else {
-#pragma unroll
-                    for (int g = 0; g < 16; ++g)
-                        if (n0 + 8 * g < p.N)
-                            *reinterpret_cast<uint4 *>(yrow + 16 * g) =
-                                make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
-                }
-            }
-            if (fused) {
-#pragma unroll
-                for (int q4 = 0; q4 < 2; ++q4) {  // two groups of 4 blocks (64 columns)
-                    uint32_t sf_word = 0;
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        const int bi = 4 * q4 + b;  // block within the 128 columns
-                        const int64_t nblk = (n0 >> 4) + bi;
-                        const bool ok_blk = row_ok && nblk < nb_y;
-                        const uint4 v0 = make_uint4(pk[8 * bi], pk[8 * bi + 1], pk[8 * bi + 2],
-                                                    pk[8 * bi + 3]);
-                        const uint4 v1 = make_uint4(pk[8 * bi + 4], pk[8 * bi + 5],
-                                                    pk[8 * bi + 6], pk[8 * bi + 7]);
-                        const uint32_t mb = max(absmax_bf16x8(v0), absmax_bf16x8(v1));
-                        const BlockScale bs = block_scale(__uint_as_float(mb << 16), s_enc_y);
-                        if (ok_blk) {
-                            amax_bits = max(amax_bits, mb);
-                            *reinterpret_cast<uint2 *>(p.yq + m * (p.N / 2) + nblk * 8) =
-                                make_uint2(quantize_bf16x8(v0, bs.inv),
-                                           quantize_bf16x8(v1, bs.inv));
-                        }
-                        sf_word |= (ok_blk ? bs.sf : 0u) << (8 * b);
-                    }
-                    const int64_t nblk0 = (n0 >> 4) + 4 * q4;
-                    if (nblk0 < nb4_y * 4)
-                        *reinterpret_cast<uint32_t *>(p.ysf + sf_offset(m, nblk0, nb4_y)) = sf_word;
-                }
-            }
+            if (lane == 0) mbar_arrive_relaxed(&acc_empty[acc]);
+            store_row_128(p, pk, int64_t(tc.m_blk) * kBM + row_in_tile,
+                          int64_t(tc.n_blk) * Cfg::BN + col0, s_enc_y, amax_bits);
         }
-        if (fused && p.amax_y != nullptr) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-                amax_bits = max(amax_bits, __shfl_xor_sync(0xFFFFFFFFu, amax_bits, o));
-            if (lane == 0 && amax_bits != 0)
-                atomicMax(reinterpret_cast<unsigned *>(p.amax_y), amax_bits << 16);
-        }
+        flush_amax_y(p, amax_bits, lane);
     }
 
     // ------------------------------------------------------------------ teardown
@@ -484,14 +397,22 @@ static cudaError_t launch_cfg(const CUtensorMap &ta, const CUtensorMap &tb, cons
 using Cfg128 = GemmConfig<128, 6, 2>;
 using Cfg256 = GemmConfig<256, 4, 1>;
 
-int gemm_tile_n(int64_t M, int64_t N) {
-    (void)M;
-    return N >= 256 ? 256 : 128;
+GemmKind gemm_kind(int64_t M, int64_t N) {
+    if (N < 256) return kGemm128;
+    // CTA pairs need at least two 128-row blocks of A to be worth it.
+    return M > 128 ? kGemmPair : kGemm256;
 }
 
+}  // namespace nvfp4
+
+#include "gemm_pair.cuh"
+
+namespace nvfp4 {
+
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
-                        int tile_n, int num_sms, cudaStream_t stream) {
-    if (tile_n == 256) return launch_cfg<Cfg256>(ta, tb, p, num_sms, stream);
+                        GemmKind kind, int num_sms, cudaStream_t stream) {
+    if (kind == kGemmPair) return launch_pair(ta, tb, p, num_sms, stream);
+    if (kind == kGemm256) return launch_cfg<Cfg256>(ta, tb, p, num_sms, stream);
     return launch_cfg<Cfg128>(ta, tb, p, num_sms, stream);
 }
 

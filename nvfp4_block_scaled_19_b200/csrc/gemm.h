@@ -20,17 +20,23 @@ struct GemmParams {
     float *amax_y;          // fused quantize: 1 fp32 (pre-zeroed) or null
     int64_t M, N, K;
     int64_t n_sf_blocks;    // ceil(N / 128): 128-row blocks present in bsf
+    int64_t m_sf_blocks;    // ceil(M / 128): 128-row blocks present in asf
 };
 
 // Device address of the library's error word (int[2]: code, tag) on the
 // current device, for kernels outside the GEMM translation unit.
 int *device_error_word();
 
-// Tile width (128 or 256) used for a problem.
-int gemm_tile_n(int64_t M, int64_t N);
+// Kernel variant for a problem: 1-CTA 128x128 tiles, 1-CTA 128x256 tiles,
+// or CTA pairs with 256x256 tiles.
+enum GemmKind { kGemm128 = 1, kGemm256 = 2, kGemmPair = 3 };
+GemmKind gemm_kind(int64_t M, int64_t N);
+
+// Rows of the B (weight) TMA box for a kernel variant.
+inline uint32_t gemm_b_box_rows(GemmKind k) { return k == kGemm256 ? 256u : 128u; }
 
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
-                        int tile_n, int num_sms, cudaStream_t stream);
+                        GemmKind kind, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_amax(const void *x, int64_t numel, float *amax, int num_sms,
                         cudaStream_t stream);

@@ -1,0 +1,125 @@
+// Pieces shared by the 1-CTA and CTA-pair block-scaled FP4 GEMM kernels:
+// the tile order and the epilogue (accumulator drain, bf16 output, optional
+// fused next-layer NVFP4 quantization of Y).
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "gemm.h"
+#include "nvfp4_math.cuh"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+struct TileCoord {
+    int m_blk, n_blk;
+};
+
+// Tile t -> (m, n) block, walking groups of kGroupM row-blocks with m fastest
+// inside a group, so concurrently running CTAs share B (weight) tiles and a
+// group's A rows stay in L2.
+constexpr int kGroupM = 8;
+__device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n) {
+    const int per_group = kGroupM * tiles_n;
+    const int g = t / per_group;
+    const int first_m = g * kGroupM;
+    const int gsz = min(tiles_m - first_m, kGroupM);
+    const int r = t - g * per_group;
+    TileCoord c;
+    c.m_blk = first_m + r % gsz;
+    c.n_blk = r / gsz;
+    return c;
+}
+
+// Reads 128 fp32 accumulator columns of this warp's 32 TMEM lanes (taddr =
+// lane base + first column), scales by alpha and rounds to packed bf16x2.
+// Two 32-column loads are in flight at a time.
+__device__ __forceinline__ void cvt_32(const uint32_t (&r)[32], float alpha, uint32_t *pk) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
+                                                       __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
+        pk[i] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+}
+
+__device__ __forceinline__ void drain_128(uint32_t taddr, float alpha, uint32_t (&pk)[64]) {
+#pragma unroll
+    for (int ch = 0; ch < 4; ch += 2) {
+        uint32_t r0[32], r1[32];
+        tmem_ld_32x32b_x32(taddr + ch * 32, r0);
+        tmem_ld_32x32b_x32(taddr + ch * 32 + 32, r1);
+        tmem_ld_wait();
+        cvt_32(r0, alpha, pk + 16 * ch);
+        cvt_32(r1, alpha, pk + 16 * ch + 16);
+    }
+}
+
+// Writes one row's 128 bf16 outputs (columns n0..n0+127 of row m) and, when
+// the GEMM fuses the next layer's quantization, its codes and block scales
+// (blocks of 16 along N with S_enc = s_enc_y).  Rows at or beyond M write no
+// Y and no codes; rows in [M, pad128(M)) write zero scales (the layout's
+// padding); rows beyond that write nothing.
+__device__ __forceinline__ void store_row_128(const GemmParams &p, const uint32_t (&pk)[64],
+                                              int64_t m, int64_t n0, float s_enc_y,
+                                              uint32_t &amax_bits) {
+    const bool row_ok = m < p.M;
+    if (row_ok && p.y != nullptr) {
+        uint8_t *yrow = p.y + (m * p.N + n0) * 2;
+        if (n0 + 128 <= p.N && (p.N & 15) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 31) == 0) {
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+                stg256(yrow + 32 * g, pk[8 * g], pk[8 * g + 1], pk[8 * g + 2], pk[8 * g + 3],
+                       pk[8 * g + 4], pk[8 * g + 5], pk[8 * g + 6], pk[8 * g + 7]);
+        } else {
+#pragma unroll
+            for (int g = 0; g < 16; ++g)
+                if (n0 + 8 * g < p.N)
+                    *reinterpret_cast<uint4 *>(yrow + 16 * g) =
+                        make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
+        }
+    }
+    if (p.yq == nullptr) return;
+    const int64_t rows_pad = (p.M + 127) & ~int64_t(127);
+    if (m >= rows_pad) return;
+    const int64_t nb_y = p.N / 16;
+    const int64_t nb4_y = (nb_y + 3) / 4;
+#pragma unroll
+    for (int q4 = 0; q4 < 2; ++q4) {  // two groups of 4 blocks (64 columns)
+        uint32_t sf_word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int bi = 4 * q4 + b;  // block within the 128 columns
+            const int64_t nblk = (n0 >> 4) + bi;
+            const bool ok_blk = row_ok && nblk < nb_y;
+            const uint4 v0 = make_uint4(pk[8 * bi], pk[8 * bi + 1], pk[8 * bi + 2], pk[8 * bi + 3]);
+            const uint4 v1 =
+                make_uint4(pk[8 * bi + 4], pk[8 * bi + 5], pk[8 * bi + 6], pk[8 * bi + 7]);
+            const uint32_t mb = max(absmax_bf16x8(v0), absmax_bf16x8(v1));
+            const BlockScale bs = block_scale(__uint_as_float(mb << 16), s_enc_y);
+            if (ok_blk) {
+                amax_bits = max(amax_bits, mb);
+                *reinterpret_cast<uint2 *>(p.yq + m * (p.N / 2) + nblk * 8) =
+                    make_uint2(quantize_bf16x8(v0, bs.inv), quantize_bf16x8(v1, bs.inv));
+            }
+            sf_word |= (ok_blk ? bs.sf : 0u) << (8 * b);
+        }
+        const int64_t nblk0 = (n0 >> 4) + 4 * q4;
+        if (nblk0 < nb4_y * 4)
+            *reinterpret_cast<uint32_t *>(p.ysf + sf_offset(m, nblk0, nb4_y)) = sf_word;
+    }
+}
+
+// Warp-reduces the fused output's |Y| maximum and folds it into amax_y.
+__device__ __forceinline__ void flush_amax_y(const GemmParams &p, uint32_t amax_bits, int lane) {
+    if (p.yq == nullptr || p.amax_y == nullptr) return;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        amax_bits = max(amax_bits, __shfl_xor_sync(0xFFFFFFFFu, amax_bits, o));
+    if (lane == 0 && amax_bits != 0)
+        atomicMax(reinterpret_cast<unsigned *>(p.amax_y), amax_bits << 16);
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,364 @@
+// Block-scaled FP4 GEMM on CTA pairs (tcgen05 cta_group::2), 256 x 256 tiles.
+//
+// Same computation as gemm_kernel (see gemm.cu), with each tile computed by
+// a cluster of two CTAs on two SMs: CTA r holds rows 128r..128r+127 of the
+// tile's A slice and rows 128r..128r+127 of its B slice in its own shared
+// memory, and one 256x256x64 MMA issued by the pair leader (CTA 0) reads both
+// CTAs' halves, leaving rows 128r..128r+127 of the accumulator in CTA r's
+// tensor memory.  Per SM this loads A 16 KB + B 16 KB per 256-element
+// k-stage for 128x256 outputs, a third less L2 -> SM traffic than the 1-CTA
+// 128x256 tile (A 16 KB + B 32 KB), which measured bound at ~20 TB/s.
+//
+// Roles (both CTAs unless noted):
+//   warp 0     producer: waits its own `empty` ring slot; the leader arms its
+//              `full` barrier with both CTAs' A+B bytes; each CTA issues
+//              `.cta_group::2` TMA loads (no multicast) of its A and B halves
+//              into its own shared memory that complete on the leader's
+//              `full` barrier, and bulk-copies its scale factors (its 128 A
+//              rows, all 256 B rows) against its own `sfload` barrier.
+//   warp 1     leader only: issues the MMAs (cta_group::2) and commits to the
+//              `empty`, `acc_full` barriers of both CTAs (tcgen05.commit
+//              multicast); both CTAs' warp 1 allocate / free the TMEM pair.
+//   warps 2-5  scale factors into this CTA's TMEM (tcgen05.st), then arrive
+//              on the leader's `sf_full` barrier (remote for CTA 1).
+//   warps 6-13 epilogue of this CTA's 128 rows; arrive on the leader's
+//              `acc_empty` barrier once the accumulator is read.
+// The scale-factor TMEM layout per CTA is the 1-CTA N = 256 one: SFA for its
+// own 128 rows, SFB for all 256 B rows, replicated in every lane quadrant.
+#pragma once
+
+namespace nvfp4 {
+
+template <int STAGES_>
+struct PairConfig {
+    static constexpr int STAGES = STAGES_;
+    static constexpr int BN = 256;  // tile columns (B rows), split 128 per CTA
+    static constexpr int BM = 256;  // tile rows, split 128 per CTA
+    static constexpr int SF_WARPS = 4;
+    static constexpr int EPI_WARPS = 8;
+    static constexpr int FIRST_SF_WARP = 2;
+    static constexpr int FIRST_EPI_WARP = FIRST_SF_WARP + SF_WARPS;
+    static constexpr int THREADS = 32 * (FIRST_EPI_WARP + EPI_WARPS);
+    static constexpr int A_BYTES = 128 * kBKBytes;
+    static constexpr int B_BYTES = 128 * kBKBytes;
+    static constexpr int SFA_BYTES = 2048;
+    static constexpr int SFB_BYTES = 4096;
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+    static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+    // full, sfload, sf_full, empty per stage; acc_full, acc_empty, drain
+    static constexpr int NUM_BARS = 4 * STAGES + 3;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+    static constexpr int SFA_COLS = 16;
+    static constexpr int SFB_COLS = 32;
+    static constexpr int SLOT_COLS = SFA_COLS + SFB_COLS;
+    static constexpr int SF_BASE = BN;  // one 256-column accumulator
+    static constexpr int TMEM_USED = SF_BASE + STAGES * SLOT_COLS;
+    static constexpr int TMEM_COLS = 512;
+    static_assert(TMEM_USED <= 512, "TMEM budget");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static constexpr uint32_t IDESC = make_idesc_mxf4nvf4(256, 256);
+};
+
+template <class Cfg>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                     const __grid_constant__ CUtensorMap tmap_b, const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
+    uint64_t *full = bars;
+    uint64_t *sfload = bars + Cfg::STAGES;
+    uint64_t *sf_full = bars + 2 * Cfg::STAGES;
+    uint64_t *empty = bars + 3 * Cfg::STAGES;
+    uint64_t *acc_full = bars + 4 * Cfg::STAGES;
+    uint64_t *acc_empty = acc_full + 1;
+    uint64_t *drain = acc_full + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + Cfg::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Cfg::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int tiles_m = static_cast<int>((p.M + Cfg::BM - 1) / Cfg::BM);
+    const int tiles_n = static_cast<int>((p.N + Cfg::BN - 1) / Cfg::BN);
+    const int num_tiles = tiles_m * tiles_n;
+    const int pair = blockIdx.x >> 1;
+    const int n_pairs = gridDim.x >> 1;
+    const int k_stages = static_cast<int>((p.K + kBK - 1) / kBK);
+    const int64_t kb4 = p.K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&sfload[s], 1);
+            mbar_init(&sf_full[s], 2 * Cfg::SF_WARPS);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 2 * Cfg::EPI_WARPS);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_b);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_holder, Cfg::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // barrier inits of both CTAs visible before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint64_t pol_a = policy_evict_normal();
+            const uint64_t pol_b = policy_evict_last();
+            const uint32_t full0 = mapa_shared(smem_addr(&full[0]), 0);  // leader's full[0]
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int t = pair; t < num_tiles && ok; t += n_pairs) {
+                const TileCoord tc = tile_coord(t, tiles_m, tiles_n);
+                const int a_row = tc.m_blk * Cfg::BM + static_cast<int>(rank) * 128;
+                const int b_row = tc.n_blk * Cfg::BN + static_cast<int>(rank) * 128;
+                const int64_t sfa_blk = int64_t(tc.m_blk) * 2 + rank;
+                const bool sfa_ok = sfa_blk < p.m_sf_blocks;
+                for (int ks = 0; ks < k_stages; ++ks) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, 11)) {
+                        ok = false;
+                        break;
+                    }
+                    const int nsub = min(4, static_cast<int>((p.K - int64_t(ks) * kBK) / 64));
+                    if (leader)
+                        mbar_arrive_expect_tx(&full[stage], 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
+                    uint32_t sf_bytes = sfa_ok ? nsub * 512 : 0;
+#pragma unroll
+                    for (int rb = 0; rb < 2; ++rb)
+                        if (int64_t(tc.n_blk) * 2 + rb < p.n_sf_blocks) sf_bytes += nsub * 512;
+                    mbar_arrive_expect_tx(&sfload[stage], sf_bytes);
+                    const uint32_t full_l = full0 + stage * 8;
+                    tma_load_2d_pair(&tmap_a, full_l, smem + Cfg::OFF_A + stage * Cfg::A_BYTES,
+                                     ks * kBKBytes, a_row, pol_a);
+                    tma_load_2d_pair(&tmap_b, full_l, smem + Cfg::OFF_B + stage * Cfg::B_BYTES,
+                                     ks * kBKBytes, b_row, pol_b);
+                    if (sfa_ok)
+                        bulk_load(smem + Cfg::OFF_SFA + stage * Cfg::SFA_BYTES,
+                                  p.asf + (sfa_blk * kb4 + int64_t(ks) * 4) * 512, nsub * 512,
+                                  &sfload[stage], pol_a);
+#pragma unroll
+                    for (int rb = 0; rb < 2; ++rb) {
+                        const int64_t brow = int64_t(tc.n_blk) * 2 + rb;
+                        if (brow < p.n_sf_blocks)
+                            bulk_load(smem + Cfg::OFF_SFB + stage * Cfg::SFB_BYTES + rb * 2048,
+                                      p.bsf + (brow * kb4 + int64_t(ks) * 4) * 512, nsub * 512,
+                                      &sfload[stage], pol_b);
+                    }
+                    if (issued < Cfg::STAGES) ++issued;
+                    if (++stage == Cfg::STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            if (!ok) {
+                // Drain this CTA's in-flight scale copies (and, on the leader,
+                // both CTAs' operand copies) with bounded waits.
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < issued; ++i) {
+                    if (--s < 0) {
+                        s = Cfg::STAGES - 1;
+                        ph ^= 1;
+                    }
+                    mbar_wait_drain(&sfload[s], ph);
+                    if (leader) mbar_wait_drain(&full[s], ph);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (leader && lane == 0) {
+            const uint64_t adesc0 = make_smem_desc(smem_addr(smem + Cfg::OFF_A), 16, 1024, 2);
+            const uint64_t bdesc0 = make_smem_desc(smem_addr(smem + Cfg::OFF_B), 16, 1024, 2);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int local = 0;
+            for (int t = pair; t < num_tiles && ok; t += n_pairs, ++local) {
+                if (!mbar_wait(acc_empty, (local & 1) ^ 1, abort_flag, 12)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int ks = 0; ks < k_stages; ++ks) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag, 13) ||
+                        !mbar_wait(&sf_full[stage], phase, abort_flag, 14)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nsub = min(4, static_cast<int>((p.K - int64_t(ks) * kBK) / 64));
+                    const uint64_t adesc = adesc0 + static_cast<uint64_t>((stage * Cfg::A_BYTES) >> 4);
+                    const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((stage * Cfg::B_BYTES) >> 4);
+                    const uint32_t sfa_t = tmem_base + Cfg::SF_BASE + stage * Cfg::SLOT_COLS;
+                    const uint32_t sfb_t = sfa_t + Cfg::SFA_COLS;
+                    for (int j = 0; j < nsub; ++j)
+                        mma_mxf4nvf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, Cfg::IDESC,
+                                          sfa_t + 4 * j, sfb_t + 8 * j,
+                                          (ks > 0 || j > 0) ? 1u : 0u);
+                    tc_commit_pair(&empty[stage], 0x3);
+                    if (++stage == Cfg::STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                tc_commit_pair(acc_full, 0x3);
+            }
+            tc_commit_pair(drain, 0x3);
+        }
+        __syncwarp();
+    } else if (warp < Cfg::FIRST_EPI_WARP) {
+        // ---------------------------------------------------------------- scale factors
+        const uint32_t lane_base = tmem_base + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
+        const uint32_t ssfa0 = smem_addr(smem + Cfg::OFF_SFA) + lane * 16;
+        const uint32_t ssfb0 = smem_addr(smem + Cfg::OFF_SFB) + lane * 16;
+        const uint32_t sf_full0 = mapa_shared(smem_addr(&sf_full[0]), 0);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int t = pair; t < num_tiles && ok; t += n_pairs) {
+            for (int ks = 0; ks < k_stages; ++ks) {
+                if (!mbar_wait_warp(&sfload[stage], phase, abort_flag, 15)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t slot = lane_base + Cfg::SF_BASE + stage * Cfg::SLOT_COLS;
+                uint32_t va[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 v = lds128(ssfa0 + stage * Cfg::SFA_BYTES + 512 * j);
+                    va[4 * j] = v.x;
+                    va[4 * j + 1] = v.y;
+                    va[4 * j + 2] = v.z;
+                    va[4 * j + 3] = v.w;
+                }
+                tmem_st_32x32b_x16(slot, va);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    // B scale column 8j + 4rb + c: MMA step j, 128-row block rb.
+                    uint32_t vb[16];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int col = 16 * h + 4 * q;
+                        const int j = col / 8;
+                        const int rb = (col / 4) % 2;
+                        const uint4 v =
+                            lds128(ssfb0 + stage * Cfg::SFB_BYTES + rb * 2048 + 512 * j);
+                        vb[4 * q] = v.x;
+                        vb[4 * q + 1] = v.y;
+                        vb[4 * q + 2] = v.z;
+                        vb[4 * q + 3] = v.w;
+                    }
+                    tmem_st_32x32b_x16(slot + Cfg::SFA_COLS + 16 * h, vb);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster_relaxed(sf_full0 + stage * 8);
+                if (++stage == Cfg::STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int e = warp - Cfg::FIRST_EPI_WARP;
+        const int quad = warp & 3;
+        const int col0 = (e >> 2) * 128;
+        const int row_in_tile = static_cast<int>(rank) * 128 + quad * 32 + lane;
+        const float alpha = __fmul_rn(*p.a_s_dec, *p.b_s_dec);
+        const float s_enc_y = p.yq != nullptr ? *p.s_enc_y : 1.0f;
+        const uint32_t acc_empty_l = mapa_shared(smem_addr(acc_empty), 0);
+        uint32_t amax_bits = 0;
+        int local = 0;
+        for (int t = pair; t < num_tiles; t += n_pairs, ++local) {
+            const TileCoord tc = tile_coord(t, tiles_m, tiles_n);
+            if (!mbar_wait_warp(acc_full, local & 1, abort_flag, 16)) break;
+            tc_fence_after();
+            uint32_t pk[64];
+            drain_128(tmem_base + col0 + ((static_cast<uint32_t>(quad) * 32) << 16), alpha, pk);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_l);
+            store_row_128(p, pk, int64_t(tc.m_blk) * Cfg::BM + row_in_tile,
+                          int64_t(tc.n_blk) * Cfg::BN + col0, s_enc_y, amax_bits);
+        }
+        flush_amax_y(p, amax_bits, lane);
+    }
+
+    // ------------------------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    if (leader && warp == 1 && *abort_flag) {
+        if (lane == 0) mbar_wait_drain(drain, 0);
+        __syncwarp();
+    }
+    // Neither CTA leaves while the pair's MMAs may still read its shared
+    // memory or a remote arrive may still target it.
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+using PairCfg = PairConfig<5>;
+
+inline cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
+                               int num_sms, cudaStream_t stream) {
+    static int configured[64] = {0};
+    static int max_clusters[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
+        e = cudaFuncSetAttribute(gemm_pair_kernel<PairCfg>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (num_sms / 2));
+        cfg.blockDim = dim3(PairCfg::THREADS);
+        cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<PairCfg>, &cfg);
+        if (e != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = num_sms / 2;
+        }
+        max_clusters[dev] = n;
+        configured[dev] = 1;
+    }
+    const int64_t tiles = ((p.M + 255) / 256) * ((p.N + 255) / 256);
+    int64_t pairs = max_clusters[dev];
+    if (pairs > tiles) pairs = tiles;
+    gemm_pair_kernel<PairCfg><<<static_cast<unsigned>(2 * pairs), PairCfg::THREADS,
+                                PairCfg::SMEM_BYTES, stream>>>(ta, tb, p);
+    return cudaGetLastError();
+}
+
+}  // namespace nvfp4
