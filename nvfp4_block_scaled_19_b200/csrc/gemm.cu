@@ -23,7 +23,9 @@
 //   warps 2-5     scale-factor warps: each copies the stage's scale factors
 //                 from shared memory into its 32-lane quadrant of TMEM with
 //                 tcgen05.st (the MMA reads every quadrant's copy), keeping
-//                 tcgen05.cp off the MMA issue stream.
+//                 tcgen05.cp off the MMA issue stream, then arrives on the
+//                 stage's `full` barrier: the MMA thread waits once per stage
+//                 for operands (TMA bytes) and scales (these arrivals) alike.
 //   warps 6..     epilogue, two warps per TMEM quadrant for BN = 256: drain
 //                 the accumulator into registers (alpha scaling, bf16
 //                 rounding), hand TMEM back to the MMA warp, then store Y and
@@ -92,7 +94,7 @@ struct GemmConfig {
     static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
     static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
-    // full, sf_full, empty per stage; acc_full, acc_empty per accumulator; drain
+    // full, sfload, empty per stage; acc_full, acc_empty per accumulator; drain
     static constexpr int NUM_BARS = 3 * STAGES + 2 * ACC_STAGES + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024 alignment
@@ -117,7 +119,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     uint64_t *full = bars;
-    uint64_t *sf_full = bars + Cfg::STAGES;
+    uint64_t *sfload = bars + Cfg::STAGES;
     uint64_t *empty = bars + 2 * Cfg::STAGES;
     uint64_t *acc_full = bars + 3 * Cfg::STAGES;
     uint64_t *acc_empty = acc_full + Cfg::ACC_STAGES;
@@ -135,8 +137,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&sf_full[s], Cfg::SF_WARPS);
+            mbar_init(&full[s], 1 + Cfg::SF_WARPS);  // producer + scale-factor warps
+            mbar_init(&sfload[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < Cfg::ACC_STAGES; ++a) {
@@ -182,21 +184,21 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
                     for (int rb = 0; rb < Cfg::NB; ++rb)
                         if (int64_t(tc.n_blk) * Cfg::NB + rb < p.n_sf_blocks) sfb_bytes += nsub * 512;
-                    mbar_arrive_expect_tx(&full[stage],
-                                          Cfg::A_BYTES + Cfg::B_BYTES + nsub * 512 + sfb_bytes);
+                    mbar_arrive_expect_tx(&full[stage], Cfg::A_BYTES + Cfg::B_BYTES);
+                    mbar_arrive_expect_tx(&sfload[stage], nsub * 512 + sfb_bytes);
                     tma_load_2d(&tmap_a, &full[stage], smem + Cfg::OFF_A + stage * Cfg::A_BYTES,
                                 ks * kBKBytes, tc.m_blk * kBM, pol_a);
                     tma_load_2d(&tmap_b, &full[stage], smem + Cfg::OFF_B + stage * Cfg::B_BYTES,
                                 ks * kBKBytes, tc.n_blk * Cfg::BN, pol_b);
                     bulk_load(smem + Cfg::OFF_SFA + stage * Cfg::SFA_BYTES, asf + ks * 2048,
-                              nsub * 512, &full[stage], pol_a);
+                              nsub * 512, &sfload[stage], pol_a);
 #pragma unroll
                     for (int rb = 0; rb < Cfg::NB; ++rb) {
                         const int64_t brow = int64_t(tc.n_blk) * Cfg::NB + rb;
                         if (brow < p.n_sf_blocks)
                             bulk_load(smem + Cfg::OFF_SFB + stage * Cfg::SFB_BYTES + rb * 2048,
                                       p.bsf + (brow * kb4 + int64_t(ks) * 4) * 512, nsub * 512,
-                                      &full[stage], pol_b);
+                                      &sfload[stage], pol_b);
                     }
                     if (issued < Cfg::STAGES) ++issued;
                     if (++stage == Cfg::STAGES) {
@@ -207,6 +209,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             }
             if (!ok) {
                 // Drain: the last `issued` stages may still be receiving data.
+                // One bounded deadline for all of them (`full` may also miss
+                // scale-warp arrivals that will never come).
+                const uint64_t deadline = globaltimer() + kWaitTimeoutNs;
                 int s = stage;
                 uint32_t ph = phase;
                 for (int i = 0; i < issued; ++i) {
@@ -214,7 +219,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                         s = Cfg::STAGES - 1;
                         ph ^= 1;
                     }
-                    mbar_wait_drain(&full[s], ph);
+                    mbar_wait_until(&sfload[s], ph, deadline);
+                    mbar_wait_until(&full[s], ph, deadline);
                 }
             }
         }
@@ -223,6 +229,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if (lane == 0) {
             const uint64_t adesc0 = make_smem_desc(smem_addr(smem + Cfg::OFF_A), 16, 1024, 2);
             const uint64_t bdesc0 = make_smem_desc(smem_addr(smem + Cfg::OFF_B), 16, 1024, 2);
+            const int k_full = static_cast<int>(p.K / kBK);          // stages of 4 MMAs
+            const int k_tail = static_cast<int>((p.K % kBK) / 64);  // MMAs in a last short stage
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -236,34 +244,49 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * Cfg::BN;
-                for (int ks = 0; ks < k_stages; ++ks) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag, 3) ||
-                        !mbar_wait(&sf_full[stage], phase, abort_flag, 5)) {
+                // Full 256-element stages: one wait, four MMAs, one commit.
+                for (int ks = 0; ks < k_full; ++ks) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag, 3)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int nsub = min(4, static_cast<int>((p.K - int64_t(ks) * kBK) / 64));
                     const uint64_t adesc = adesc0 + static_cast<uint64_t>((stage * Cfg::A_BYTES) >> 4);
                     const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((stage * Cfg::B_BYTES) >> 4);
                     const uint32_t sfa_t = tmem_base + Cfg::SF_BASE + stage * Cfg::SLOT_COLS;
                     const uint32_t sfb_t = sfa_t + Cfg::SFA_COLS;
-                    if (nsub == 4) {
+                    mma_mxf4nvf4(d_tmem, adesc, bdesc, Cfg::IDESC, sfa_t, sfb_t, ks > 0 ? 1u : 0u);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            mma_mxf4nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, Cfg::IDESC,
-                                         sfa_t + 4 * j, sfb_t + 4 * Cfg::NB * j,
-                                         (ks > 0 || j > 0) ? 1u : 0u);
-                    } else {
-                        for (int j = 0; j < nsub; ++j)
-                            mma_mxf4nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, Cfg::IDESC,
-                                         sfa_t + 4 * j, sfb_t + 4 * Cfg::NB * j,
-                                         (ks > 0 || j > 0) ? 1u : 0u);
-                    }
+                    for (int j = 1; j < 4; ++j)
+                        mma_mxf4nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, Cfg::IDESC,
+                                     sfa_t + 4 * j, sfb_t + 4 * Cfg::NB * j, 1u);
                     tc_commit(&empty[stage]);
                     if (++stage == Cfg::STAGES) {
                         stage = 0;
                         phase ^= 1;
+                    }
+                }
+                if (ok && k_tail > 0) {
+                    // Last stage of a K that is not a multiple of 256.
+                    if (!mbar_wait(&full[stage], phase, abort_flag, 5)) {
+                        ok = false;
+                    } else {
+                        tc_fence_after();
+                        const uint64_t adesc =
+                            adesc0 + static_cast<uint64_t>((stage * Cfg::A_BYTES) >> 4);
+                        const uint64_t bdesc =
+                            bdesc0 + static_cast<uint64_t>((stage * Cfg::B_BYTES) >> 4);
+                        const uint32_t sfa_t = tmem_base + Cfg::SF_BASE + stage * Cfg::SLOT_COLS;
+                        const uint32_t sfb_t = sfa_t + Cfg::SFA_COLS;
+                        for (int j = 0; j < k_tail; ++j)
+                            mma_mxf4nvf4(d_tmem, adesc + 2 * j, bdesc + 2 * j, Cfg::IDESC,
+                                         sfa_t + 4 * j, sfb_t + 4 * Cfg::NB * j,
+                                         (k_full > 0 || j > 0) ? 1u : 0u);
+                        tc_commit(&empty[stage]);
+                        if (++stage == Cfg::STAGES) {
+                            stage = 0;
+                            phase ^= 1;
+                        }
                     }
                 }
                 if (!ok) break;
@@ -287,7 +310,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         bool ok = true;
         for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
             for (int ks = 0; ks < k_stages; ++ks) {
-                if (!mbar_wait_warp(&full[stage], phase, abort_flag, 6)) {
+                if (!mbar_wait_warp(&sfload[stage], phase, abort_flag, 6)) {
                     ok = false;
                     break;
                 }
@@ -324,7 +347,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_relaxed(&sf_full[stage]);
+                if (lane == 0) mbar_arrive_relaxed(&full[stage]);
                 if (++stage == Cfg::STAGES) {
                     stage = 0;
                     phase ^= 1;

@@ -48,12 +48,15 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, const flo
 // Workspace of the single-launch dynamic quantization (zero-initialised once
 // by the caller; calls that share one must be stream-ordered).
 struct DynWorkspace {
+    // (barrier generation << 32) | amax bits of the launch that completed it;
+    // one 64-bit word, so a CTA leaving the grid barrier reads both at once.
+    unsigned long long state;
     unsigned count;         // CTAs arrived at the grid barrier (back to 0 after it)
-    unsigned gen;           // barrier generation, +1 per launch
-    unsigned amax_bits[2];  // amax of launch g in [g & 1]; the other is cleared
-    float fallback_amax;    // used when rows are too wide for one cooperative grid
+    unsigned amax_acc;      // running amax bits of the current launch (back to 0 after it)
+    float fallback_amax;    // used when rows are too wide for one resident grid
     unsigned pad[3];
 };
+static_assert(sizeof(DynWorkspace) == 32, "workspace size is part of the ABI");
 
 // Returns cudaErrorNotSupported when the rows are too wide for one
 // cooperative grid (then use launch_amax + launch_quantize).

@@ -20,11 +20,18 @@
 //              `empty`, `acc_full` barriers of both CTAs (tcgen05.commit
 //              multicast); both CTAs' warp 1 allocate / free the TMEM pair.
 //   warps 2-5  scale factors into this CTA's TMEM (tcgen05.st), then arrive
-//              on the leader's `sf_full` barrier (remote for CTA 1).
+//              on the leader's `full` barrier (remote for CTA 1), so that one
+//              wait per stage covers operands and scales alike.
 //   warps 6-13 epilogue of this CTA's 128 rows; arrive on the leader's
 //              `acc_empty` barrier once the accumulator is read.
 // The scale-factor TMEM layout per CTA is the 1-CTA N = 256 one: SFA for its
 // own 128 rows, SFB for all 256 B rows, replicated in every lane quadrant.
+//
+// The MMA issue loop is the critical path: the tensor pipe queues only about
+// two MMAs, so the issuing thread has roughly 256 cycles between MMAs for its
+// own work.  Measured on B200, one barrier wait plus the commit fits, a second
+// wait per stage or a loop over a run-time number of MMAs does not; hence the
+// single `full` barrier and the fully unrolled stage body.
 #pragma once
 
 namespace nvfp4 {
@@ -48,8 +55,8 @@ struct PairConfig {
     static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
     static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
-    // full, sfload, sf_full, empty per stage; acc_full, acc_empty, drain
-    static constexpr int NUM_BARS = 4 * STAGES + 3;
+    // full, sfload, empty per stage; acc_full, acc_empty, drain
+    static constexpr int NUM_BARS = 3 * STAGES + 3;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
     static constexpr int SFA_COLS = 16;
@@ -73,9 +80,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::OFF_BAR);
     uint64_t *full = bars;
     uint64_t *sfload = bars + Cfg::STAGES;
-    uint64_t *sf_full = bars + 2 * Cfg::STAGES;
-    uint64_t *empty = bars + 3 * Cfg::STAGES;
-    uint64_t *acc_full = bars + 4 * Cfg::STAGES;
+    uint64_t *empty = bars + 2 * Cfg::STAGES;
+    uint64_t *acc_full = bars + 3 * Cfg::STAGES;
     uint64_t *acc_empty = acc_full + 1;
     uint64_t *drain = acc_full + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + Cfg::OFF_MISC);
@@ -95,9 +101,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            // The leader's producer arrival (with both CTAs' operand bytes)
+            // plus every scale-factor warp of the pair.
+            mbar_init(&full[s], 1 + 2 * Cfg::SF_WARPS);
             mbar_init(&sfload[s], 1);
-            mbar_init(&sf_full[s], 2 * Cfg::SF_WARPS);
             mbar_init(&empty[s], 1);
         }
         mbar_init(acc_full, 1);
@@ -175,7 +182,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
             }
             if (!ok) {
                 // Drain this CTA's in-flight scale copies (and, on the leader,
-                // both CTAs' operand copies) with bounded waits.
+                // both CTAs' operand copies) under one bounded deadline; `full`
+                // may also miss scale-warp arrivals that will never come.
+                const uint64_t deadline = globaltimer() + kWaitTimeoutNs;
                 int s = stage;
                 uint32_t ph = phase;
                 for (int i = 0; i < issued; ++i) {
@@ -183,8 +192,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                         s = Cfg::STAGES - 1;
                         ph ^= 1;
                     }
-                    mbar_wait_drain(&sfload[s], ph);
-                    if (leader) mbar_wait_drain(&full[s], ph);
+                    mbar_wait_until(&sfload[s], ph, deadline);
+                    if (leader) mbar_wait_until(&full[s], ph, deadline);
                 }
             }
         }
@@ -193,6 +202,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         if (leader && lane == 0) {
             const uint64_t adesc0 = make_smem_desc(smem_addr(smem + Cfg::OFF_A), 16, 1024, 2);
             const uint64_t bdesc0 = make_smem_desc(smem_addr(smem + Cfg::OFF_B), 16, 1024, 2);
+            const int k_full = static_cast<int>(p.K / kBK);          // stages of 4 MMAs
+            const int k_tail = static_cast<int>((p.K % kBK) / 64);  // MMAs in a last short stage
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -203,26 +214,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                for (int ks = 0; ks < k_stages; ++ks) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag, 13) ||
-                        !mbar_wait(&sf_full[stage], phase, abort_flag, 14)) {
+                // Full 256-element stages: one wait, four MMAs, one commit.
+                for (int ks = 0; ks < k_full; ++ks) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag, 13)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int nsub = min(4, static_cast<int>((p.K - int64_t(ks) * kBK) / 64));
                     const uint64_t adesc = adesc0 + static_cast<uint64_t>((stage * Cfg::A_BYTES) >> 4);
                     const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((stage * Cfg::B_BYTES) >> 4);
                     const uint32_t sfa_t = tmem_base + Cfg::SF_BASE + stage * Cfg::SLOT_COLS;
                     const uint32_t sfb_t = sfa_t + Cfg::SFA_COLS;
-                    for (int j = 0; j < nsub; ++j)
+                    mma_mxf4nvf4_pair(tmem_base, adesc, bdesc, Cfg::IDESC, sfa_t, sfb_t,
+                                      ks > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int j = 1; j < 4; ++j)
                         mma_mxf4nvf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, Cfg::IDESC,
-                                          sfa_t + 4 * j, sfb_t + 8 * j,
-                                          (ks > 0 || j > 0) ? 1u : 0u);
+                                          sfa_t + 4 * j, sfb_t + 8 * j, 1u);
                     tc_commit_pair(&empty[stage], 0x3);
                     if (++stage == Cfg::STAGES) {
                         stage = 0;
                         phase ^= 1;
+                    }
+                }
+                if (ok && k_tail > 0) {
+                    // Last stage of a K that is not a multiple of 256.
+                    if (!mbar_wait(&full[stage], phase, abort_flag, 14)) {
+                        ok = false;
+                    } else {
+                        tc_fence_after();
+                        const uint64_t adesc =
+                            adesc0 + static_cast<uint64_t>((stage * Cfg::A_BYTES) >> 4);
+                        const uint64_t bdesc =
+                            bdesc0 + static_cast<uint64_t>((stage * Cfg::B_BYTES) >> 4);
+                        const uint32_t sfa_t = tmem_base + Cfg::SF_BASE + stage * Cfg::SLOT_COLS;
+                        const uint32_t sfb_t = sfa_t + Cfg::SFA_COLS;
+                        for (int j = 0; j < k_tail; ++j)
+                            mma_mxf4nvf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, Cfg::IDESC,
+                                              sfa_t + 4 * j, sfb_t + 8 * j,
+                                              (k_full > 0 || j > 0) ? 1u : 0u);
+                        tc_commit_pair(&empty[stage], 0x3);
+                        if (++stage == Cfg::STAGES) {
+                            stage = 0;
+                            phase ^= 1;
+                        }
                     }
                 }
                 if (!ok) break;
@@ -236,7 +271,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         const uint32_t lane_base = tmem_base + ((static_cast<uint32_t>(warp & 3) * 32) << 16);
         const uint32_t ssfa0 = smem_addr(smem + Cfg::OFF_SFA) + lane * 16;
         const uint32_t ssfb0 = smem_addr(smem + Cfg::OFF_SFB) + lane * 16;
-        const uint32_t sf_full0 = mapa_shared(smem_addr(&sf_full[0]), 0);
+        const uint32_t full0 = mapa_shared(smem_addr(&full[0]), 0);  // leader's full[0]
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -278,7 +313,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster_relaxed(sf_full0 + stage * 8);
+                if (lane == 0) mbar_arrive_cluster_relaxed(full0 + stage * 8);
                 if (++stage == Cfg::STAGES) {
                     stage = 0;
                     phase ^= 1;

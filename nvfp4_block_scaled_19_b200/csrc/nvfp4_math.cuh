@@ -137,7 +137,9 @@ __device__ __forceinline__ uint32_t quantize_bf16x8(uint4 v, float inv) {
 
 // Byte offset of the block scale (row r, block c) in the 128x4-tiled layout
 // whose rows hold kb4 = ceil(kb/4) tiles.
-__device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t kb4) {
+// T is int64_t, or uint32_t where the caller has checked every offset < 2^31.
+template <typename T>
+__device__ __forceinline__ T sf_offset(T r, T c, T kb4) {
     return ((r >> 7) * kb4 + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
 }
 

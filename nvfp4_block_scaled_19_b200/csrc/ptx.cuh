@@ -109,6 +109,15 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) 
     }
 }
 
+// Abort-path drain of several barriers under one deadline (a %globaltimer
+// value): returns at completion or once the deadline has passed.
+__device__ __forceinline__ void mbar_wait_until(uint64_t *bar, uint32_t parity, uint64_t deadline) {
+    const uint32_t a = smem_addr(bar);
+    while (!mbar_try_wait(a, parity)) {
+        if (globaltimer() > deadline) return;
+    }
+}
+
 // ------------------------------------------------------------------ clusters (CTA pairs)
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {

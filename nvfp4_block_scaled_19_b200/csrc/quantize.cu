@@ -15,11 +15,17 @@
 //   shuffles into one 4-byte store in the 128x4-tiled layout.  The kernel also
 //   writes the layout's zero padding (rows up to a multiple of 128, blocks up
 //   to a multiple of 4), so the scale buffer needs no memset.
-// quantize_dynamic: both in one cooperative launch.  Phase 1 reduces the
-//   amax (one atomicMax per CTA into a per-launch word of a small workspace),
-//   a bounded grid barrier publishes it, phase 2 quantizes.  Phase 2 walks the
-//   rows in the opposite order to phase 1, so the part of the tensor phase 1
-//   read last is still in L2 (all of it when the tensor fits in L2).
+// quantize_dynamic: both in one launch of a grid that is resident all at
+//   once.  Phase 1 reduces the amax (one atomicMax per CTA into a per-launch
+//   word of a small workspace), a bounded grid barrier publishes it, phase 2
+//   quantizes, walking the tensor in the opposite order to phase 1 so that
+//   what phase 1 read last is still in L2 (all of it when the tensor fits).
+//   Rows of a multiple of 64 elements (every DiT shape) take the flat kernel:
+//   the tensor is seen as one array of 16-element blocks, thread g owns
+//   blocks g, g + S, g + 2S, g + 3S of each round (S = threads in the grid),
+//   so every thread has four 32-byte loads in flight in both phases and a
+//   warp's codes are one contiguous 256-byte store.  Other widths take the
+//   row-stream kernel (quantize_rows).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -161,40 +167,193 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(
 
 constexpr int kDynThreads = 512;  // 4 row streams x 128 threads
 
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_gpu(unsigned *p, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
 
-// Cooperative launch (8 row streams x 64 threads): every CTA is resident, so the grid barrier cannot
-// deadlock; it is still bounded (error tag 7 on timeout).
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Relaxed load with no compiler barrier: issued early, consumed late.
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned *p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+// Called by one thread per CTA with the CTA's amax bits (bf16 |x| pattern)
+// and the generation it read from ws->state at kernel start.  Folds the bits
+// into the launch's running amax, then waits (bounded) for every CTA.  The
+// arrival is a release-acquire RMW on the counter; the last arrival reads the
+// final amax, resets the counter and the running amax for the next launch,
+// and publishes (gen + 1, amax) with one release store that the other CTAs
+// poll, so leaving the barrier costs no further read.  Returns false (and
+// records error tag 7) on timeout.
+__device__ __forceinline__ bool grid_amax_barrier(DynWorkspace *ws, unsigned gen, uint32_t m,
+                                                  int *err, unsigned *amax_bits_out) {
+    if (m != 0) atomicMax(&ws->amax_acc, m << 16);
+    const unsigned arrived = atom_add_acq_rel_gpu(&ws->count, 1u);
+    if (arrived == gridDim.x - 1) {
+        const unsigned a = *reinterpret_cast<volatile unsigned *>(&ws->amax_acc);
+        ws->count = 0u;  // both resets are ordered before the release below
+        ws->amax_acc = 0u;
+        st_release_gpu_u64(&ws->state, (static_cast<unsigned long long>(gen + 1) << 32) | a);
+        *amax_bits_out = a;
+        return true;
+    }
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        const unsigned long long st = ld_acquire_gpu_u64(&ws->state);
+        if (static_cast<unsigned>(st >> 32) != gen) {
+            *amax_bits_out = static_cast<unsigned>(st);
+            return true;
+        }
+        if (globaltimer_ns() - t0 > kBarrierTimeoutNs) {
+            if (err != nullptr && atomicCAS(err, 0, 5) == 0) err[1] = 7;
+            return false;
+        }
+        __nanosleep(32);
+    }
+}
+
+constexpr int kFlatThreads = 512;
+constexpr int kFlatU = 4;  // 16-element blocks (32-byte loads) in flight per thread
+
+// Flat dynamic quantization for cols % 64 == 0 (so 4 consecutive blocks never
+// straddle a row and the scale layout has no column padding).  Block v of the
+// tensor (row v / kb, block column v % kb) is the 32 bytes at x + 32 v; its
+// codes are the 8 bytes at q + 8 v.  Idx is uint32_t when the block count and
+// the grid's index range fit 32 bits (register pressure), else int64_t.
+template <typename Idx>
+__global__ void __launch_bounds__(kFlatThreads, 2) quantize_dynamic_flat_kernel(
+    const uint8_t *__restrict__ x, int64_t rows, int64_t cols, uint8_t *__restrict__ q,
+    uint8_t *__restrict__ sf, float *__restrict__ s_dec_out, float *__restrict__ amax_out,
+    DynWorkspace *ws, int *err) {
+    __shared__ unsigned s_amax;
+    __shared__ int s_fail;
+    __shared__ uint32_t red[kFlatThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // Only thread 0 needs the generation; its load overlaps phase 1's.  The
+    // previous launch on this workspace has completed (stream order).
+    const unsigned long long state0 = tid == 0 ? ld_relaxed_gpu_u64(&ws->state) : 0ull;
+
+    const bool a32 = (reinterpret_cast<uintptr_t>(x) & 31) == 0;
+    const Idx kb = static_cast<Idx>(cols >> 4);
+    const Idx kb4 = kb >> 2;
+    const Idx nvec = static_cast<Idx>(rows) * kb;  // a multiple of 4
+    const Idx S = static_cast<Idx>(gridDim.x) * kFlatThreads;
+    const Idx chunk = S * kFlatU;
+    const Idx g = static_cast<Idx>(blockIdx.x) * kFlatThreads + tid;
+    const Idx n_rounds = (nvec + chunk - 1) / chunk;
+
+    auto load_round = [&](Idx rd, BF16x16 (&v)[kFlatU]) {
+#pragma unroll
+        for (int u = 0; u < kFlatU; ++u) {
+            const Idx idx = rd * chunk + u * S + g;
+            if (idx < nvec) {
+                v[u] = ldg_32B(x + 32 * static_cast<int64_t>(idx), a32);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[u].w[k] = 0u;
+            }
+        }
+    };
+
+    // Phase 1: amax.  v keeps the last round for phase 2.
+    uint32_t m = 0;
+    BF16x16 v[kFlatU];
+    for (Idx rd = 0; rd < n_rounds; ++rd) {
+        load_round(rd, v);
+#pragma unroll
+        for (int u = 0; u < kFlatU; ++u) m = max(m, absmax_bf16x16(v[u]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    if (warp == 0) {
+        m = lane < kFlatThreads / 32 ? red[lane] : 0u;
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane == 0) {
+            unsigned bits = 0;
+            s_fail = grid_amax_barrier(ws, static_cast<unsigned>(state0 >> 32), m, err, &bits) ? 0 : 1;
+            s_amax = bits;
+        }
+    }
+    __syncthreads();
+    if (s_fail) return;
+    const float amax = __uint_as_float(s_amax);
+    const float s_enc = tensor_encode_scale(amax);
+    if (blockIdx.x == 0 && tid == 0) {
+        if (s_dec_out != nullptr) *s_dec_out = __fdiv_rn(1.0f, s_enc);
+        if (amax_out != nullptr) *amax_out = amax;
+    }
+
+    // Phase 2: quantize, rounds in reverse order (the last round straight
+    // from the registers phase 1 left it in).  Validity is uniform over
+    // each group of 4 lanes (nvec and every warp's first index are multiples
+    // of 4), so the scale gather's shuffles see consistent neighbours.
+    for (Idx rd = n_rounds; rd-- > 0;) {
+        if (rd + 1 != n_rounds) load_round(rd, v);
+#pragma unroll
+        for (int u = 0; u < kFlatU; ++u) {
+            const Idx idx = rd * chunk + u * S + g;
+            const bool valid = idx < nvec;
+            const BlockScale bs = block_scale(__uint_as_float(absmax_bf16x16(v[u]) << 16), s_enc);
+            if (valid) {
+                const uint4 lo = make_uint4(v[u].w[0], v[u].w[1], v[u].w[2], v[u].w[3]);
+                const uint4 hi = make_uint4(v[u].w[4], v[u].w[5], v[u].w[6], v[u].w[7]);
+                *reinterpret_cast<uint2 *>(q + 8 * static_cast<int64_t>(idx)) =
+                    make_uint2(quantize_bf16x8(lo, bs.inv), quantize_bf16x8(hi, bs.inv));
+            }
+            const uint32_t sfc = valid ? bs.sf : 0u;
+            const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sfc, 1);
+            const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sfc, 2);
+            const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sfc, 3);
+            if (valid && (lane & 3) == 0) {
+                const Idx r = idx / kb;
+                const Idx c = idx - r * kb;
+                *reinterpret_cast<uint32_t *>(sf + sf_offset(r, c, kb4)) =
+                    sfc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            }
+        }
+    }
+    // Zero scales of the padding rows [rows, pad128(rows)).
+    const Idx rows_i = static_cast<Idx>(rows);
+    const Idx n_pad = (((rows_i + 127) & ~Idx(127)) - rows_i) * kb4;
+    for (Idx i = g; i < n_pad; i += S) {
+        const Idx pr = i / kb4;
+        *reinterpret_cast<uint32_t *>(sf + sf_offset(rows_i + pr, 4 * (i - pr * kb4), kb4)) = 0u;
+    }
+}
+
+// Row-stream variant (8 row streams x 64 threads) for widths that are not a
+// multiple of 64.  The grid is resident all at once; the barrier is bounded.
 __global__ void __launch_bounds__(kDynThreads) quantize_dynamic_kernel(
     const uint16_t *__restrict__ x, int64_t rows, int64_t cols, uint8_t *__restrict__ q,
     uint8_t *__restrict__ sf, float *__restrict__ s_dec_out, float *__restrict__ amax_out,
     DynWorkspace *ws, int *err, int gx) {
-    __shared__ unsigned s_gen, s_amax;
+    __shared__ unsigned s_amax;
     __shared__ int s_fail;
     __shared__ uint32_t red[kDynThreads / 32];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid == 0) {
-        s_gen = ld_acquire_gpu(&ws->gen);
-        s_fail = 0;
-    }
-    __syncthreads();
-    const unsigned gen = s_gen;
-    // The next launch's amax word starts at zero; nobody reads it in this one.
-    if (blockIdx.x == 0 && tid == 0) ws->amax_bits[(gen + 1) & 1] = 0u;
+    const unsigned long long state0 = tid == 0 ? ld_relaxed_gpu_u64(&ws->state) : 0ull;
 
     // Phase 1: amax (32-byte loads, four in flight per thread).
     const uint8_t *xb = reinterpret_cast<const uint8_t *>(x);
@@ -221,27 +380,9 @@ __global__ void __launch_bounds__(kDynThreads) quantize_dynamic_kernel(
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
         if (lane == 0) {
-            if (m != 0) atomicMax(&ws->amax_bits[gen & 1], m << 16);
-            __threadfence();
-            // Grid barrier: the last CTA to arrive resets the count and
-            // advances the generation; the others wait for that.
-            const unsigned arrived = atomicAdd(&ws->count, 1u);
-            if (arrived == gridDim.x - 1) {
-                ws->count = 0u;
-                __threadfence();
-                st_release_gpu(&ws->gen, gen + 1);
-            } else {
-                const uint64_t t0 = globaltimer_ns();
-                while (ld_acquire_gpu(&ws->gen) == gen) {
-                    if (globaltimer_ns() - t0 > kBarrierTimeoutNs) {
-                        s_fail = 1;
-                        if (err != nullptr && atomicCAS(err, 0, 5) == 0) err[1] = 7;
-                        break;
-                    }
-                    __nanosleep(64);
-                }
-            }
-            s_amax = ld_acquire_gpu(&ws->amax_bits[gen & 1]);
+            unsigned bits = 0;
+            s_fail = grid_amax_barrier(ws, static_cast<unsigned>(state0 >> 32), m, err, &bits) ? 0 : 1;
+            s_amax = bits;
         }
     }
     __syncthreads();
@@ -309,29 +450,59 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, const flo
 cudaError_t launch_quantize_dynamic(const void *x, int64_t rows, int64_t cols, uint8_t *q,
                                     uint8_t *sf, float *s_dec_out, float *amax_out,
                                     DynWorkspace *ws, int num_sms, cudaStream_t stream) {
-    static int resident[64] = {0};
+    static int resident_rows[64] = {0};
+    static int resident_flat[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (resident[dev] == 0) {
+    const bool flat = cols % 64 == 0;
+    int &resident = flat ? resident_flat[dev] : resident_rows[dev];
+    if (resident == 0) {
         int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_dynamic_kernel,
-                                                          kDynThreads, 0);
+        // Both index widths of the flat kernel have the same launch bounds.
+        e = flat ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                       &per_sm, quantize_dynamic_flat_kernel<int64_t>, kFlatThreads, 0)
+                 : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quantize_dynamic_kernel,
+                                                                 kDynThreads, 0);
         if (e != cudaSuccess || per_sm < 1) return e != cudaSuccess ? e : cudaErrorInvalidValue;
-        resident[dev] = per_sm;
+        resident = per_sm;
+    }
+    int grid = num_sms * resident;
+    int *err = device_error_word();
+    // The grid barrier needs every CTA resident at once: the grid is exactly
+    // what the occupancy query says fits, and the launch is cooperative, so
+    // the runtime guarantees it (or refuses the launch).
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(flat ? kFlatThreads : kDynThreads);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (flat) {
+        cfg.gridDim = dim3(grid);
+        const uint8_t *xb = reinterpret_cast<const uint8_t *>(x);
+        // 32-bit indices when every index the kernel forms (blocks, padded
+        // scale offsets, the last round's overshoot) stays below 2^31.
+        const int64_t nvec = rows * (cols / 16);
+        const int64_t span = int64_t(grid) * kFlatThreads * kFlatU;
+        const int64_t sf_span = ((rows + 127) / 128 * 128) * (cols / 16);
+        if (nvec + span < (int64_t(1) << 31) && sf_span < (int64_t(1) << 31))
+            return cudaLaunchKernelEx(&cfg, quantize_dynamic_flat_kernel<uint32_t>, xb, rows, cols,
+                                      q, sf, s_dec_out, amax_out, ws, err);
+        return cudaLaunchKernelEx(&cfg, quantize_dynamic_flat_kernel<int64_t>, xb, rows, cols, q,
+                                  sf, s_dec_out, amax_out, ws, err);
     }
     const int64_t kbp = ((cols / 16 + 3) / 4) * 4;
     int gx = static_cast<int>((kbp + kSliceBlocks - 1) / kSliceBlocks);
-    int grid = num_sms * resident[dev];
     // Phase 2 needs at least one CTA per column slice; very wide rows use
-    // several passes of the slices (not reached by DiT shapes).
+    // the two-kernel path instead.
     if (gx > grid) return cudaErrorNotSupported;
     grid = (grid / gx) * gx;
-    int *err = device_error_word();
-    const uint16_t *xp = reinterpret_cast<const uint16_t *>(x);
-    void *args[] = {&xp, &rows, &cols, &q, &sf, &s_dec_out, &amax_out, &ws, &err, &gx};
-    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(quantize_dynamic_kernel),
-                                       dim3(grid), dim3(kDynThreads), args, 0, stream);
+    cfg.gridDim = dim3(grid);
+    return cudaLaunchKernelEx(&cfg, quantize_dynamic_kernel, reinterpret_cast<const uint16_t *>(x),
+                              rows, cols, q, sf, s_dec_out, amax_out, ws, err, gx);
 }
 
 }  // namespace nvfp4

@@ -28,8 +28,10 @@ def test_amax(nv, orc, numel):
     assert np.float32(amax.item()) == want
 
 
+# Widths that are multiples of 64 take the flat single-launch kernel, the
+# others the row-stream one; both appear, with ragged row counts.
 SMALL_SHAPES = [(1, 16), (3, 48), (127, 80), (128, 64), (130, 272), (257, 512), (64, 3072),
-                (1000, 16), (5, 4096)]
+                (1000, 16), (5, 4096), (1, 64), (129, 192)]
 
 
 PATHS = ["two_kernel", "fused"]
@@ -83,14 +85,15 @@ def _edge_tensor(kind, rows=130, cols=80):
     raise ValueError(kind)
 
 
+@pytest.mark.parametrize("cols", [80, 128])
 @pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("kind", ["zeros", "negative_zeros", "mixed_zero_blocks",
                                   "bf16_subnormals", "subnormals_with_zeros", "huge",
                                   "underflow_blocks", "one_hot", "ties"])
-def test_quantize_edge_cases(nv, kind, path):
-    x = _edge_tensor(kind)
+def test_quantize_edge_cases(nv, kind, path, cols):
+    x = _edge_tensor(kind, cols=cols)
     assert_quant_equal(gpu_quantize_dynamic(nv, x, path), oracle_quantize_dynamic(x),
-                       f"{kind}/{path}")
+                       f"{kind}/{path}/{cols}")
 
 
 def test_quantize_dynamic_back_to_back(nv):
@@ -133,11 +136,12 @@ def test_quantize_workloads_full_size(nv, name):
         del x, wt
 
 
+@pytest.mark.parametrize("cols", [272, 320])
 @pytest.mark.parametrize("path", PATHS)
-def test_quantize_input_16_byte_aligned(nv, path):
+def test_quantize_input_16_byte_aligned(nv, path, cols):
     """An input that is 16-byte but not 32-byte aligned (a view 8 elements
     into a buffer) takes the two-load path and gives the same codes."""
-    rows, cols = 130, 272
+    rows = 130
     x = draw_x("normal_outliers", rows, cols, seed=77, index=0)
     buf = torch.zeros(rows * cols + 16, dtype=torch.bfloat16, device="cuda")
     view = buf[8:8 + rows * cols].view(rows, cols)
