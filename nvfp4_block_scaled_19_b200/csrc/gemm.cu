@@ -97,7 +97,8 @@ struct GemmConfig {
     // full, sfload, empty per stage; acc_full, acc_empty per accumulator; drain
     static constexpr int NUM_BARS = 3 * STAGES + 2 * ACC_STAGES + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024 alignment
+    static constexpr int OFF_INV = OFF_MISC + 16;  // 128-entry block-multiplier table
+    static constexpr int SMEM_BYTES = OFF_INV + 512 + 1024;  // + slack for 1024 alignment
     // TMEM columns: accumulators, then one scale-factor slot per stage.
     static constexpr int SFA_COLS = 16;       // 4 MMAs x 4 columns (128 rows)
     static constexpr int SFB_COLS = 16 * NB;  // 4 MMAs x 4*NB columns
@@ -157,6 +158,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         tmem_alloc(tmem_holder, Cfg::TMEM_COLS);
         tmem_relinquish();
     }
+    float *inv_tab = reinterpret_cast<float *>(smem + Cfg::OFF_INV);
+    if (p.yq != nullptr) fill_inv_table(inv_tab, *p.s_enc_y);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -372,14 +375,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             tc_fence_after();
             // Drain 128 accumulator columns into 64 packed bf16x2 registers.
             uint32_t pk[64];
-            drain_128(tmem_base + acc * Cfg::BN + col0 + ((static_cast<uint32_t>(quad) * 32) << 16),
+            drain_cols<128>(tmem_base + acc * Cfg::BN + col0 + ((static_cast<uint32_t>(quad) * 32) << 16),
                       alpha, pk);
             // Accumulator read: hand it back to the MMA warp.
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_relaxed(&acc_empty[acc]);
-            store_row_128(p, pk, int64_t(tc.m_blk) * kBM + row_in_tile,
-                          int64_t(tc.n_blk) * Cfg::BN + col0, s_enc_y, amax_bits);
+            store_row<128>(p, pk, int64_t(tc.m_blk) * kBM + row_in_tile,
+                          int64_t(tc.n_blk) * Cfg::BN + col0, s_enc_y, inv_tab, amax_bits);
         }
         flush_amax_y(p, amax_bits, lane);
     }

@@ -33,9 +33,9 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n)
     return c;
 }
 
-// Reads 128 fp32 accumulator columns of this warp's 32 TMEM lanes (taddr =
-// lane base + first column), scales by alpha and rounds to packed bf16x2.
-// Two 32-column loads are in flight at a time.
+// Reads NC (64 or 128) fp32 accumulator columns of this warp's 32 TMEM lanes
+// (taddr = lane base + first column), scales by alpha and rounds to packed
+// bf16x2.  Two 32-column loads are in flight at a time.
 __device__ __forceinline__ void cvt_32(const uint32_t (&r)[32], float alpha, uint32_t *pk) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -45,9 +45,11 @@ __device__ __forceinline__ void cvt_32(const uint32_t (&r)[32], float alpha, uin
     }
 }
 
-__device__ __forceinline__ void drain_128(uint32_t taddr, float alpha, uint32_t (&pk)[64]) {
+template <int NC>
+__device__ __forceinline__ void drain_cols(uint32_t taddr, float alpha, uint32_t (&pk)[NC / 2]) {
+    static_assert(NC == 64 || NC == 128, "64 or 128 columns");
 #pragma unroll
-    for (int ch = 0; ch < 4; ch += 2) {
+    for (int ch = 0; ch < NC / 32; ch += 2) {
         uint32_t r0[32], r1[32];
         tmem_ld_32x32b_x32(taddr + ch * 32, r0);
         tmem_ld_32x32b_x32(taddr + ch * 32 + 32, r1);
@@ -57,25 +59,26 @@ __device__ __forceinline__ void drain_128(uint32_t taddr, float alpha, uint32_t 
     }
 }
 
-// Writes one row's 128 bf16 outputs (columns n0..n0+127 of row m) and, when
-// the GEMM fuses the next layer's quantization, its codes and block scales
-// (blocks of 16 along N with S_enc = s_enc_y).  Rows at or beyond M write no
-// Y and no codes; rows in [M, pad128(M)) write zero scales (the layout's
-// padding); rows beyond that write nothing.
-__device__ __forceinline__ void store_row_128(const GemmParams &p, const uint32_t (&pk)[64],
-                                              int64_t m, int64_t n0, float s_enc_y,
-                                              uint32_t &amax_bits) {
+// Writes one row's NC (64 or 128) bf16 outputs (columns n0..n0+NC-1 of row
+// m) and, when the GEMM fuses the next layer's quantization, their codes and
+// block scales (blocks of 16 along N with S_enc = s_enc_y).  Rows at or
+// beyond M write no Y and no codes; rows in [M, pad128(M)) write zero scales
+// (the layout's padding); rows beyond that write nothing.
+template <int NC>
+__device__ __forceinline__ void store_row(const GemmParams &p, const uint32_t (&pk)[NC / 2],
+                                          int64_t m, int64_t n0, float s_enc_y,
+                                          const float *inv_tab, uint32_t &amax_bits) {
     const bool row_ok = m < p.M;
     if (row_ok && p.y != nullptr) {
         uint8_t *yrow = p.y + (m * p.N + n0) * 2;
-        if (n0 + 128 <= p.N && (p.N & 15) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 31) == 0) {
+        if (n0 + NC <= p.N && (p.N & 15) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 31) == 0) {
 #pragma unroll
-            for (int g = 0; g < 8; ++g)
+            for (int g = 0; g < NC / 16; ++g)
                 stg256(yrow + 32 * g, pk[8 * g], pk[8 * g + 1], pk[8 * g + 2], pk[8 * g + 3],
                        pk[8 * g + 4], pk[8 * g + 5], pk[8 * g + 6], pk[8 * g + 7]);
         } else {
 #pragma unroll
-            for (int g = 0; g < 16; ++g)
+            for (int g = 0; g < NC / 8; ++g)
                 if (n0 + 8 * g < p.N)
                     *reinterpret_cast<uint4 *>(yrow + 16 * g) =
                         make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
@@ -87,18 +90,18 @@ __device__ __forceinline__ void store_row_128(const GemmParams &p, const uint32_
     const int64_t nb_y = p.N / 16;
     const int64_t nb4_y = (nb_y + 3) / 4;
 #pragma unroll
-    for (int q4 = 0; q4 < 2; ++q4) {  // two groups of 4 blocks (64 columns)
+    for (int q4 = 0; q4 < NC / 64; ++q4) {  // groups of 4 blocks (64 columns)
         uint32_t sf_word = 0;
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-            const int bi = 4 * q4 + b;  // block within the 128 columns
+            const int bi = 4 * q4 + b;  // block within the NC columns
             const int64_t nblk = (n0 >> 4) + bi;
             const bool ok_blk = row_ok && nblk < nb_y;
             const uint4 v0 = make_uint4(pk[8 * bi], pk[8 * bi + 1], pk[8 * bi + 2], pk[8 * bi + 3]);
             const uint4 v1 =
                 make_uint4(pk[8 * bi + 4], pk[8 * bi + 5], pk[8 * bi + 6], pk[8 * bi + 7]);
             const uint32_t mb = max(absmax_bf16x8(v0), absmax_bf16x8(v1));
-            const BlockScale bs = block_scale(__uint_as_float(mb << 16), s_enc_y);
+            const BlockScale bs = block_scale(__uint_as_float(mb << 16), s_enc_y, inv_tab);
             if (ok_blk) {
                 amax_bits = max(amax_bits, mb);
                 *reinterpret_cast<uint2 *>(p.yq + m * (p.N / 2) + nblk * 8) =

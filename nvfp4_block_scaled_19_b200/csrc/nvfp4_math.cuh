@@ -47,17 +47,43 @@ struct BlockScale {
     float inv;    // multiplier taking x to E2M1 code space
 };
 
-__device__ __forceinline__ BlockScale block_scale(float a_b, float s_enc) {
-    const float s = __fmul_rn(__fdiv_rn(a_b, 6.0f), s_enc);
+// RN_fp32(a / 6) for every bf16 value a (subnormals included), computed as
+// the double product a * RN64(1/6) rounded once to fp32.  Why it equals the
+// IEEE fp32 quotient: a = M * 2^k with k >= -133, so a / 6 measured in units
+// of its fp32 ulp (or of the subnormal spacing 2^-149) is an integer multiple
+// of 1/3: it lies 0, 1/3 or 2/3 of a unit above a representable value, at
+// least 1/6 unit from every rounding midpoint, while the double product is
+// within 2^-52 relative of a / 6 (far below 1/6 unit); both round to the same
+// fp32 value.  (The argument uses a's form; the fp32 product a * RN32(1/6)
+// is not enough and differs for thousands of bf16 values.)
+__device__ __forceinline__ float div6_short(float a) {
+    return __double2float_rn(static_cast<double>(a) * (1.0 / 6.0));
+}
+
+// The block multiplier S_enc / sf depends only on the launch's S_enc and the
+// 8-bit E4M3 code, so each CTA tabulates it once for the 127 finite
+// non-negative codes (cvt ... satfinite never yields 0x7F):
+//   inv[c] = sf_c == 0 ? 0 : min(S_enc / sf_c, FLT_MAX)   (IEEE division)
+// Called by all threads of the CTA; the caller syncs before use.
+__device__ __forceinline__ void fill_inv_table(float *tab, float s_enc) {
+    for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+        const float sfv = e4m3_decode(static_cast<uint32_t>(c));
+        float inv = 0.0f;
+        if (sfv != 0.0f) {
+            inv = __fdiv_rn(s_enc, sfv);
+            if (!isfinite(inv)) inv = FLT_MAX;
+        }
+        tab[c] = inv;
+    }
+}
+
+// Block scale of a 16-element block with amax a_b (a bf16 value):
+//   s = (a_b / 6) * S_enc ; sf = E4M3_rn_satfinite(s) ; inv = tab[sf]
+__device__ __forceinline__ BlockScale block_scale(float a_b, float s_enc, const float *inv_tab) {
+    const float s = __fmul_rn(div6_short(a_b), s_enc);
     BlockScale b;
     b.sf = e4m3_encode(s);
-    const float sfv = e4m3_decode(b.sf);
-    float inv = 0.0f;
-    if (sfv != 0.0f) {
-        inv = __fdiv_rn(s_enc, sfv);
-        if (!isfinite(inv)) inv = FLT_MAX;
-    }
-    b.inv = inv;
+    b.inv = inv_tab[b.sf];
     return b;
 }
 

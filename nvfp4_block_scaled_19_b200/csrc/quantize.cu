@@ -85,9 +85,10 @@ constexpr int kQuantRows = 2;       // rows per group; the next group is loaded 
 // rows up to a multiple of 128 and block columns up to a multiple of 4 get
 // zero scales.  All 32 lanes of a warp share (bx, rs), so shuffles are uniform.
 __device__ __forceinline__ void quantize_rows(const uint16_t *__restrict__ x, int64_t rows,
-                                              int64_t cols, float s_enc, uint8_t *__restrict__ q,
-                                              uint8_t *__restrict__ sf, int bx, int64_t rs,
-                                              int64_t n_streams, int tx, bool descending) {
+                                              int64_t cols, float s_enc, const float *inv_tab,
+                                              uint8_t *__restrict__ q, uint8_t *__restrict__ sf,
+                                              int bx, int64_t rs, int64_t n_streams, int tx,
+                                              bool descending) {
     const int64_t kb = cols >> 4;
     const int64_t kb4 = (kb + 3) >> 2;  // scale tiles per 128-row block
     const int64_t kbp = kb4 << 2;       // padded blocks per row
@@ -128,7 +129,8 @@ __device__ __forceinline__ void quantize_rows(const uint16_t *__restrict__ x, in
             const int64_t r = r0 + u;
             if (r >= rows_pad) break;  // uniform across the warp
             const bool valid = r < rows && col_ok;
-            const BlockScale bs = block_scale(__uint_as_float(absmax_bf16x16(cur[u]) << 16), s_enc);
+            const BlockScale bs =
+                block_scale(__uint_as_float(absmax_bf16x16(cur[u]) << 16), s_enc, inv_tab);
             const uint32_t sfc = valid ? bs.sf : 0u;
             if (valid) {
                 const uint4 lo = make_uint4(cur[u].w[0], cur[u].w[1], cur[u].w[2], cur[u].w[3]);
@@ -159,8 +161,11 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(
     const float s_enc = kDynamic ? tensor_encode_scale(*scale_in) : *scale_in;
     if (s_dec_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
         *s_dec_out = __fdiv_rn(1.0f, s_enc);
+    __shared__ float inv_tab[128];
+    fill_inv_table(inv_tab, s_enc);
+    __syncthreads();
     constexpr int kStreams = kQuantThreads / kSliceBlocks;
-    quantize_rows(x, rows, cols, s_enc, q, sf, blockIdx.x,
+    quantize_rows(x, rows, cols, s_enc, inv_tab, q, sf, blockIdx.x,
                   static_cast<int64_t>(blockIdx.y) * kStreams + threadIdx.x / kSliceBlocks,
                   static_cast<int64_t>(gridDim.y) * kStreams, threadIdx.x % kSliceBlocks, false);
 }
@@ -247,6 +252,7 @@ __global__ void __launch_bounds__(kFlatThreads, 2) quantize_dynamic_flat_kernel(
     __shared__ unsigned s_amax;
     __shared__ int s_fail;
     __shared__ uint32_t red[kFlatThreads / 32];
+    __shared__ float inv_tab[128];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // Only thread 0 needs the generation; its load overlaps phase 1's.  The
     // previous launch on this workspace has completed (stream order).
@@ -304,6 +310,8 @@ __global__ void __launch_bounds__(kFlatThreads, 2) quantize_dynamic_flat_kernel(
         if (s_dec_out != nullptr) *s_dec_out = __fdiv_rn(1.0f, s_enc);
         if (amax_out != nullptr) *amax_out = amax;
     }
+    fill_inv_table(inv_tab, s_enc);
+    __syncthreads();
 
     // Phase 2: quantize, rounds in reverse order (the last round straight
     // from the registers phase 1 left it in).  Validity is uniform over
@@ -315,7 +323,8 @@ __global__ void __launch_bounds__(kFlatThreads, 2) quantize_dynamic_flat_kernel(
         for (int u = 0; u < kFlatU; ++u) {
             const Idx idx = rd * chunk + u * S + g;
             const bool valid = idx < nvec;
-            const BlockScale bs = block_scale(__uint_as_float(absmax_bf16x16(v[u]) << 16), s_enc);
+            const BlockScale bs =
+                block_scale(__uint_as_float(absmax_bf16x16(v[u]) << 16), s_enc, inv_tab);
             if (valid) {
                 const uint4 lo = make_uint4(v[u].w[0], v[u].w[1], v[u].w[2], v[u].w[3]);
                 const uint4 hi = make_uint4(v[u].w[4], v[u].w[5], v[u].w[6], v[u].w[7]);
@@ -352,6 +361,7 @@ __global__ void __launch_bounds__(kDynThreads) quantize_dynamic_kernel(
     __shared__ unsigned s_amax;
     __shared__ int s_fail;
     __shared__ uint32_t red[kDynThreads / 32];
+    __shared__ float inv_tab[128];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned long long state0 = tid == 0 ? ld_relaxed_gpu_u64(&ws->state) : 0ull;
 
@@ -393,13 +403,15 @@ __global__ void __launch_bounds__(kDynThreads) quantize_dynamic_kernel(
         if (s_dec_out != nullptr) *s_dec_out = __fdiv_rn(1.0f, s_enc);
         if (amax_out != nullptr) *amax_out = amax;
     }
+    fill_inv_table(inv_tab, s_enc);
+    __syncthreads();
 
     // Phase 2: quantize, rows descending.
     const int nby = static_cast<int>(gridDim.x) / gx;
     const int byc = static_cast<int>(blockIdx.x) / gx;
     if (byc >= nby) return;
     constexpr int kStreams = kDynThreads / kSliceBlocks;
-    quantize_rows(x, rows, cols, s_enc, q, sf, static_cast<int>(blockIdx.x) % gx,
+    quantize_rows(x, rows, cols, s_enc, inv_tab, q, sf, static_cast<int>(blockIdx.x) % gx,
                   static_cast<int64_t>(byc) * kStreams + tid / kSliceBlocks,
                   static_cast<int64_t>(nby) * kStreams, tid % kSliceBlocks, true);
 }
