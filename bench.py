@@ -43,6 +43,49 @@ FP4_PER_BF16 = 4.0      # nominal dense FP4 / dense BF16 (9 / 2.25 PFLOP/s)
 NOMINAL_FP4_TFLOPS = 9000.0
 
 
+GEMM_SOURCES = ["gemm.h", "gemm.cu", "gemm_pair.cuh", "gemm_common.cuh", "ptx.cuh",
+                "nvfp4_math.cuh"]
+
+
+def gemm_source_hash() -> str:
+    """sha256 over the GEMM kernel sources, in a fixed order: ties a profile's
+    counters to the kernel they were taken on."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "nvfp4_block_scaled_19_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload: str) -> tuple[float | None, str]:
+    """DRAM bytes per launch of the workload's dominant GEMM from the committed
+    ncu summary profiles/gemm_pair_<workload>.md, or None when there is none or
+    the kernel sources changed after the capture."""
+    path = os.path.join(ROOT, "profiles", f"gemm_pair_{workload}.md")
+    try:
+        with open(path) as f:
+            kv = dict(l.split(":", 1) for l in f.read().splitlines()
+                      if l.startswith(("traffic_bytes_per_launch:", "source_sha256:")))
+    except OSError:
+        return None, "no ncu summary"
+    if kv.get("source_sha256", "").strip() != gemm_source_hash():
+        return None, "kernel changed since the ncu capture"
+    try:
+        return float(kv["traffic_bytes_per_launch"]), os.path.relpath(path, ROOT)
+    except (KeyError, ValueError):
+        return None, "no traffic line"
+
+
+def gemm_kernel_name(M: int, N: int) -> str:
+    """Which kernel nvfp4_gemm dispatches to (mirrors gemm_kind in csrc/gemm.cu)."""
+    if N >= 256 and M > 128:
+        return "gemm_pair_kernel (tcgen05.mma cta_group::2 kind::mxf4nvf4, 256x256 tiles)"
+    if N >= 256:
+        return "gemm_kernel 128x256 (tcgen05.mma kind::mxf4nvf4)"
+    return "gemm_kernel 128x128 (tcgen05.mma kind::mxf4nvf4)"
+
+
 def load_peaks() -> tuple[dict, str]:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -177,6 +220,17 @@ class Layer:
         return 2 * self.M * self.N * self.K
 
     @property
+    def gemm_bytes(self) -> int:
+        """Algorithmic bytes of the GEMM: codes + scales of X and W read once,
+        Y (bf16) written once (plus the fused codes + scales when fused)."""
+        import nvfp4_block_scaled_19_b200 as nv
+        b = (self.M + self.N) * self.K // 2 + nv.sf_bytes(self.M, self.K) + nv.sf_bytes(self.N, self.K)
+        b += 2 * self.M * self.N
+        if self.fused is not None:
+            b += self.M * self.N // 2 + nv.sf_bytes(self.M, self.N)
+        return b
+
+    @property
     def quant_bytes(self) -> int:
         """Algorithmic bytes of amax (read X) + quantize (read X, write codes + scales)."""
         import nvfp4_block_scaled_19_b200 as nv
@@ -261,6 +315,7 @@ def gpu_arm(args) -> dict | None:
     q_bytes = sum(L.quant_bytes for L in layers)
     q_gbs = q_bytes / (sum(q_avg) * 1e-3) / 1e9
 
+    traffic, traffic_src = profiled_traffic(w.name)
     e2e = host_e2e(nv, layers, args, device, dist, world)
     clocks = sampler.summary()
 
@@ -286,10 +341,12 @@ def gpu_arm(args) -> dict | None:
                              "L2 where the input fits)"},
         "gemm": {"tflops": round(gemm_tflops, 1), "ms": round(g_avg[top], 5),
                  "layer": layers[top].spec.name},
-        "roofline": {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 mxf4nvf4)",
+        "roofline": {"bound": "tensor",
+                     "kernel": gemm_kernel_name(layers[top].M, layers[top].N),
                      "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
-                     "traffic": None,
+                     "traffic": traffic, "traffic_source": traffic_src,
+                     "algorithmic_bytes": layers[top].gemm_bytes,
                      "peak_source": f"{peak_src}: 4 x bf16_tflops burst ({bf16_burst}); "
                                     f"sustained would be {FP4_PER_BF16 * bf16_sust}"},
         "clocks": clocks,
@@ -297,7 +354,7 @@ def gpu_arm(args) -> dict | None:
         "gpu_launches": 2 * n_l * args.steps,
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, args.cpu_rows)
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     return line
 
 
@@ -353,15 +410,27 @@ def oracle_sample(w, rows: int) -> tuple[float, int, str]:
     return secs, flops, desc
 
 
-def cpu_baseline(w, rows: int) -> dict:
+def sample_rows(w, seconds_per_pass: float) -> int:
+    """Rows per oracle pass so that one pass takes about `seconds_per_pass`
+    (from a timed 64-row pass), between 64 and the workload's M."""
+    t64, _, _ = oracle_sample(w, 64)
+    rows = int(64 * seconds_per_pass / max(t64, 1e-6))
+    return max(64, min(w.M, rows))
+
+
+def cpu_baseline(w, target_s: float) -> dict:
+    """The oracle as it stands on the host cores: passes over a row slice of
+    the workload (all rows when they fit) until about target_s of work."""
     import oracle
     oracle.lib()
-    oracle_sample(w, min(rows, 64))       # warm-up
-    runs = [oracle_sample(w, rows) for _ in range(3)]
-    secs = statistics.median(r[0] for r in runs)
-    return {"value": round(runs[0][1] / secs / 1e12, 6), "unit": UNIT,
-            "cores": oracle.num_threads(), "kind": "oracle", "sample": runs[0][2],
-            "seconds": round(secs, 3)}
+    rows = sample_rows(w, target_s / 4)
+    secs, flops, passes, desc = 0.0, 0, 0, ""
+    while passes == 0 or secs < target_s:
+        s, f, desc = oracle_sample(w, rows)
+        secs, flops, passes = secs + s, flops + f, passes + 1
+    return {"value": round(flops / secs / 1e12, 6), "unit": UNIT,
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{passes} passes of: {desc}", "seconds": round(secs, 3)}
 
 
 def reference_arm(args) -> dict | None:
@@ -372,12 +441,13 @@ def reference_arm(args) -> dict | None:
     oracle.lib()
     w = WORKLOADS[args.workload]
     for _ in range(max(args.warmup, 1)):
-        oracle_sample(w, min(args.cpu_rows, 64))
+        oracle_sample(w, 64)
+    rows = sample_rows(w, args.cpu_seconds / 8)
     secs, flops = 0.0, 0
     desc = ""
     steps = max(1, args.steps if args.steps <= 20 else 20)
     for _ in range(steps):
-        s, f, desc = oracle_sample(w, args.cpu_rows)
+        s, f, desc = oracle_sample(w, rows)
         secs += s
         flops += f
     value = flops / secs / 1e12
@@ -401,7 +471,8 @@ def main(argv=None) -> int:
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=list(WORKLOADS), default=DEFAULT_WORKLOAD)
-    ap.add_argument("--cpu-rows", type=int, default=256)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="oracle work timed for cpu_baseline (per reference step: 1/8 of it)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

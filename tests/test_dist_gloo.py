@@ -59,4 +59,28 @@ def test_reference_arm_only_rank0_prints(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "2")
     import bench
     assert bench.reference_arm(bench.argparse.Namespace(
-        workload="tiny_linear", warmup=1, steps=1, cpu_rows=16)) is None
+        workload="tiny_linear", warmup=1, steps=1, cpu_seconds=0.1)) is None
+
+
+def test_reference_arm_rank0_line(monkeypatch):
+    """Rank 0 of the reference arm times the oracle and fills the contract's
+    keys (impl, cpu_baseline, e2e with zero copy bytes)."""
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    import bench
+    line = bench.reference_arm(bench.argparse.Namespace(
+        workload="tiny_linear", warmup=1, steps=2, cpu_seconds=0.2))
+    assert line["impl"] == "reference" and line["steps"] == 2
+    assert line["value"] > 0 and line["unit"] == bench.UNIT
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["e2e"]["value"] == line["value"]
+
+
+def test_cpu_baseline_sample_is_bounded():
+    import bench
+    from workloads import WORKLOADS
+    t0 = bench.time.perf_counter()
+    cb = bench.cpu_baseline(WORKLOADS["tiny_linear"], 0.3)
+    assert bench.time.perf_counter() - t0 < 30
+    assert cb["seconds"] >= 0.3 and cb["value"] > 0 and "passes of" in cb["sample"]
