@@ -1,11 +1,14 @@
 """Benchmark of the NVFP4 linear-layer hot path on B200.
 
 One step = one pass of the whole per-call path over one batch of synthetic
-DiT activations: for every layer of the workload, the per-tensor amax, the
-dynamic NVFP4 quantize and the block-scaled FP4 GEMM (with the fused
-next-layer quantize where the layer feeds one).  Weights are quantized once,
-before timing (static scale).  The headline metric is NVFP4 GEMM TFLOP/s
-including the activation quantize, i.e. 2*M*N*K / (t_amax + t_quantize +
+DiT activations: for every layer of the workload, the single-launch dynamic
+NVFP4 quantize of its input (amax, tensor scale, block quantize) and the
+block-scaled FP4 GEMM, with the fused next-layer quantize (and activation)
+in the GEMM epilogue where the layer feeds one; a layer whose input is the
+previous layer's fused output skips the quantize.  Weights are quantized
+once, before timing (static scale); a fused output's static tensor scale is
+calibrated once from an untimed pass.  The headline metric is NVFP4 GEMM
+TFLOP/s including the activation quantize, i.e. 2*M*N*K / (t_quantize +
 t_gemm) summed over layers.
 
 Multi-GPU: one process per GPU (torchrun); each rank runs an independent
@@ -198,22 +201,25 @@ class ClockSampler:
 # ----------------------------------------------------------------- the GPU arm
 
 class Layer:
-    def __init__(self, nv, spec, x_cpu, w_cpu, device):
+    def __init__(self, nv, spec, M, x_cpu, w_cpu, device):
         self.spec = spec
-        self.M, self.K = x_cpu.shape
+        self.M, self.K = M, spec.K
         self.N = w_cpu.shape[0]
-        self.x = x_cpu.to(device)
         self.x_cpu = x_cpu
+        self.x = None if x_cpu is None else x_cpu.to(device)
         self.lin = nv.NVFP4Linear(w_cpu.to(device))
-        self.xq = nv.empty_nvfp4(self.M, self.K, device)
+        self.xq = None if spec.x_from_prev else nv.empty_nvfp4(self.M, self.K, device)
         self.amax = torch.empty(1, dtype=torch.float32, device=device)
-        self.y = torch.empty(self.M, self.N, dtype=torch.bfloat16, device=device)
+        self.y = (torch.empty(self.M, self.N, dtype=torch.bfloat16, device=device)
+                  if spec.keep_y else None)
         self.fused = None
         if spec.fused_out:
-            # Next-layer tensor scale: static, from a calibration amax of 8.
+            # Next-layer tensor scale: static; calibrate() replaces this first
+            # guess (amax 8) with 2688 / amax of an untimed pass.
             self.fused = nv.FusedQuant(torch.tensor([2688.0 / 8.0], device=device),
                                        nv.empty_nvfp4(self.M, self.N, device),
-                                       torch.empty(1, dtype=torch.float32, device=device))
+                                       torch.empty(1, dtype=torch.float32, device=device),
+                                       nv.ACT_GELU if spec.act == "gelu" else nv.ACT_NONE)
 
     @property
     def flops(self) -> int:
@@ -232,24 +238,50 @@ class Layer:
 
     @property
     def quant_bytes(self) -> int:
-        """Algorithmic bytes of amax (read X) + quantize (read X, write codes + scales)."""
+        """Algorithmic bytes of amax (read X) + quantize (read X, write codes +
+        scales); 0 for a layer fed by the previous layer's fused output."""
         import nvfp4_block_scaled_19_b200 as nv
+        if self.spec.x_from_prev:
+            return 0
         n = self.M * self.K
         return 2 * n + 2 * n + n // 2 + nv.sf_bytes(self.M, self.K)
 
 
+def layer_input(layers, i):
+    """The quantized X of layer i: its own buffer, or the previous layer's
+    fused output."""
+    L = layers[i]
+    return layers[i - 1].fused.out if L.spec.x_from_prev else L.xq
+
+
 def run_step(nv, layers, ev=None):
-    """One pass of the hot path; ev: optional per-layer event pairs around the
-    quantize pair and the GEMM."""
+    """One pass of the hot path; ev: optional per-layer event triples around
+    the quantize and the GEMM (the quantize span is empty for a chained layer)."""
     for i, L in enumerate(layers):
         if ev is not None:
             ev[i][0].record()
-        nv.quantize_dynamic(L.x, L.xq, L.amax)
+        if not L.spec.x_from_prev:
+            nv.quantize_dynamic(L.x, L.xq, L.amax)
         if ev is not None:
             ev[i][1].record()
-        nv.gemm(L.xq, L.lin.w, L.y, L.fused)
+        nv.gemm(layer_input(layers, i), L.lin.w, L.y, L.fused, want_y=L.y is not None)
         if ev is not None:
             ev[i][2].record()
+
+
+def calibrate(nv, layers) -> None:
+    """Static tensor scales of the fused outputs: one untimed pass, then
+    S_enc = 2688 / amax of each fused output (device-side, before timing)."""
+    run_step(nv, layers)
+    for L in layers:
+        if L.fused is not None:
+            a = L.fused.amax.clamp_min(torch.finfo(torch.float32).tiny)
+            L.fused.s_enc.copy_(torch.full_like(a, 2688.0) / a)
+    torch.cuda.synchronize()
+
+
+def launches_per_step(layers) -> int:
+    return sum(1 + (0 if L.spec.x_from_prev else 1) for L in layers)
 
 
 def gpu_arm(args) -> dict | None:
@@ -261,9 +293,10 @@ def gpu_arm(args) -> dict | None:
     nv.lib()
     peaks, peak_src = load_peaks()
     w = WORKLOADS[args.workload]
-    layers = [Layer(nv, l, *layer_inputs(w, i), device) for i, l in enumerate(w.layers)]
+    layers = [Layer(nv, l, w.M, *layer_inputs(w, i), device) for i, l in enumerate(w.layers)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     torch.cuda.synchronize()
+    calibrate(nv, layers)
 
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
@@ -313,7 +346,8 @@ def gpu_arm(args) -> dict | None:
     gemm_tflops = layers[top].flops / (g_avg[top] * 1e-3) / 1e12
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     q_bytes = sum(L.quant_bytes for L in layers)
-    q_gbs = q_bytes / (sum(q_avg) * 1e-3) / 1e9
+    q_ms_sum = sum(q_avg[i] for i, L in enumerate(layers) if not L.spec.x_from_prev)
+    q_gbs = q_bytes / (q_ms_sum * 1e-3) / 1e9 if q_bytes else 0.0
 
     traffic, traffic_src = profiled_traffic(w.name)
     e2e = host_e2e(nv, layers, args, device, dist, world)
@@ -329,13 +363,15 @@ def gpu_arm(args) -> dict | None:
         "dtype": "nvfp4 (e2m1 x ue4m3 block scales, fp32 accumulate, bf16 out)",
         "data": "synthetic (seeded DiT-shaped activations and N(0,1/K) weights)",
         "config": {"workload": w.name, "description": w.description, "M": w.M,
-                   "layers": [[l.name, l.K, l.N] for l in w.layers],
+                   "layers": [[l.name, l.K, l.N] + (["gelu"] if l.act == "gelu" else [])
+                              + (["input: previous fused output"] if l.x_from_prev else [])
+                              for l in w.layers],
                    "l2": "flushed between steps (256 MiB write, outside the timed spans)",
                    "parallelism": f"replicas x{world}"},
         "pct_fp4_peak": {"of_4x_measured_bf16_burst": round(value / world / fp4_peak, 4),
                          "of_nominal_9pf": round(value / world / NOMINAL_FP4_TFLOPS, 4)},
         "quantize": {"gbs": round(q_gbs, 1), "pct_hbm": round(q_gbs / hbm, 4),
-                     "ms_per_step": round(sum(q_avg), 5),
+                     "ms_per_step": round(q_ms_sum, 5),
                      "note": "single-launch amax + dynamic quantize of every layer input; "
                              "algorithmic bytes 4.5625 B/elem + scales (second read from "
                              "L2 where the input fits)"},
@@ -351,7 +387,7 @@ def gpu_arm(args) -> dict | None:
                                     f"sustained would be {FP4_PER_BF16 * bf16_sust}"},
         "clocks": clocks,
         "e2e": e2e,
-        "gpu_launches": 2 * n_l * args.steps,
+        "gpu_launches": launches_per_step(layers) * args.steps,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
@@ -359,7 +395,12 @@ def gpu_arm(args) -> dict | None:
 
 
 def host_e2e(nv, layers, args, device, dist, world) -> dict:
-    """Same metric through nvfp4_linear_host: pinned host X in, host Y out."""
+    """Same metric end to end: pinned host X in, host Y out, copies timed.
+    Independent layers go through nvfp4_linear_host; a chain (a layer fed by
+    the previous layer's fused output) through the Python API, copying every
+    drawn X in and the last layer's Y out."""
+    if any(L.spec.x_from_prev for L in layers):
+        return chain_e2e(nv, layers, args, device, dist, world)
     stream = torch.cuda.current_stream()
     hosts = []
     for L in layers:
@@ -387,22 +428,60 @@ def host_e2e(nv, layers, args, device, dist, world) -> dict:
             "steps": steps, "api": "nvfp4_linear_host (C ABI, pinned host buffers)"}
 
 
+def chain_e2e(nv, layers, args, device, dist, world) -> dict:
+    xs = [(L, L.x_cpu.contiguous().pin_memory()) for L in layers if L.x_cpu is not None]
+    last = layers[-1]
+    yh = torch.empty(last.M, last.N, dtype=torch.bfloat16).pin_memory()
+    steps = max(1, min(args.steps, args.e2e_steps))
+
+    def one():
+        for L, xh in xs:
+            L.x.copy_(xh, non_blocking=True)
+        run_step(nv, layers)
+        yh.copy_(last.y, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    sec = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, device)
+    flops = sum(L.flops for L in layers) * steps
+    return {"value": round(aggregate(flops, world, sec) / 1e12, 3), "unit": UNIT,
+            "h2d_bytes_per_step": sum(L.M * L.K * 2 for L, _ in xs),
+            "d2h_bytes_per_step": last.M * last.N * 2, "steps": steps,
+            "api": "Python API (quantize_dynamic, gemm with fused epilogue), pinned host buffers"}
+
+
 # ----------------------------------------------------------------- CPU oracle (baseline / reference)
 
 def oracle_sample(w, rows: int) -> tuple[float, int, str]:
     """One bounded oracle pass: for every layer, amax + quantize of a `rows`-row
-    slice of X, quantize of W (its static scale), and the dequantize-then-fp64
-    GEMM of that slice. Returns (seconds, flops, description)."""
+    slice of X (for a chained layer: the previous layer's output, activated and
+    rounded to bf16, quantized with its own tensor scale), quantize of W (its
+    static scale), and the dequantize-then-fp64 GEMM of that slice.
+    Returns (seconds, flops, description)."""
+    import numpy as np
     import oracle
     from workloads import bf16_bits
     secs, flops = 0.0, 0
+    prev = None
     for li, l in enumerate(w.layers):
         x, wt = layer_inputs(w, li, M=rows)
-        xb, wb = bf16_bits(x), bf16_bits(wt)
-        bq, bsf, bsd, _ = oracle.quantize_dynamic(wb, l.N, l.K)   # static weights: untimed
+        bq, bsf, bsd, _ = oracle.quantize_dynamic(bf16_bits(wt), l.N, l.K)  # static: untimed
         t0 = time.perf_counter()
-        aq, asf, asd, _ = oracle.quantize_dynamic(xb, rows, l.K)
-        oracle.gemm(aq, asf, asd, bq, bsf, bsd, rows, l.N, l.K)
+        if l.x_from_prev:
+            xb = bf16_bits(torch.from_numpy(prev.astype(np.float32)).to(torch.bfloat16))
+            aq, asf, asd, _ = oracle.quantize_dynamic(xb, rows, l.K)
+        else:
+            aq, asf, asd, _ = oracle.quantize_dynamic(bf16_bits(x), rows, l.K)
+        y = oracle.gemm(aq, asf, asd, bq, bsf, bsd, rows, l.N, l.K)
+        prev = oracle.gelu(y) if l.act == "gelu" else y
         secs += time.perf_counter() - t0
         flops += 2 * rows * l.N * l.K
     desc = (f"{rows} rows of every layer input of {w.name} (full K, full N): amax + quantize "

@@ -66,20 +66,41 @@ typedef enum {
     NVFP4_ERR_TIMEOUT = 5
 } nvfp4_status;
 
+/* Activation applied to the GEMM output inside a fused epilogue, before the
+ * bf16 rounding.  The pages' GEMM kernels fuse consecutive operations into
+ * the GEMM (xalabuda page, section "Квантование NVFP4 и оптимизация
+ * вычислительных ядер"); in a DiT block the FFN up-projection is followed by
+ * its activation, read here as the exact (erf) GELU, whose output is the
+ * FFN down-projection's input. */
+typedef enum {
+    NVFP4_ACT_NONE = 0,
+    NVFP4_ACT_GELU = 1 /* g(h) = 0.5 h (1 + erf(h / sqrt(2))) in fp32, erf by
+                        * Abramowitz & Stegun 7.1.26 (|error| <= 1.5e-7) */
+} nvfp4_activation;
+
 /* Optional fused output quantization of the GEMM (the next layer's
- * activation quantize, done in the GEMM epilogue).  Y is first rounded to
- * bf16, then quantized in blocks of 16 along N with the caller's S_enc
- * (static, or the previous call's amax via 2688/amax).  Requires N % 16 == 0.
- *   s_enc_y  device, 1 fp32, read
- *   yq       device, M*N/2 bytes, written (packed E2M1, row-major)
- *   ysf      device, nvfp4_sf_bytes(M, N) bytes, written (tiled SF, padding 0)
- *   amax_y   device, 1 fp32, overwritten with max|Y| over the bf16 Y
- *            (NULL = not computed). */
+ * activation quantize, done in the GEMM epilogue).  With h = alpha * acc in
+ * fp32, Y = bf16_rn(h) (activation NONE) or bf16_rn(g(h)) (GELU); Y is then
+ * quantized in blocks of 16 along N with the caller's S_enc (static, or the
+ * previous call's amax via 2688/amax).  The bf16 output y_bf16 of
+ * nvfp4_gemm, when given, is this same Y.  Requires N % 16 == 0.
+ *   s_enc_y    device, 1 fp32, read
+ *   yq         device, M*N/2 bytes, written (packed E2M1, row-major)
+ *   ysf        device, nvfp4_sf_bytes(M, N) bytes, written (tiled SF, padding 0)
+ *   amax_y     device, 1 fp32, overwritten with max|Y| over the bf16 Y
+ *              (NULL = not computed)
+ *   s_dec_y    device, 1 fp32, written with 1/S_enc (IEEE fp32 division), the
+ *              decode scale a GEMM consuming (yq, ysf) needs (NULL = not
+ *              written)
+ *   activation an nvfp4_activation value; anything else is
+ *              NVFP4_ERR_INVALID_ARG */
 typedef struct {
     const float *s_enc_y;
     uint8_t *yq;
     uint8_t *ysf;
     float *amax_y;
+    float *s_dec_y;
+    int activation;
 } nvfp4_fused_out;
 
 /* Bytes of packed E2M1 data for a [rows, cols] tensor: rows * cols / 2. */

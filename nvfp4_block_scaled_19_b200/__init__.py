@@ -35,7 +35,12 @@ class NVFP4Error(RuntimeError):
 
 class FusedOut(ctypes.Structure):
     _fields_ = [("s_enc_y", ctypes.c_void_p), ("yq", ctypes.c_void_p),
-                ("ysf", ctypes.c_void_p), ("amax_y", ctypes.c_void_p)]
+                ("ysf", ctypes.c_void_p), ("amax_y", ctypes.c_void_p),
+                ("s_dec_y", ctypes.c_void_p), ("activation", ctypes.c_int)]
+
+
+ACT_NONE = 0   # nvfp4_activation values
+ACT_GELU = 1
 
 
 class LinearWorkspace(ctypes.Structure):
@@ -193,10 +198,13 @@ def quantize_dynamic(x: torch.Tensor, out: NVFP4Tensor | None = None,
 
 @dataclass
 class FusedQuant:
-    """Fused next-layer quantization outputs of a GEMM."""
+    """Fused next-layer quantization outputs of a GEMM.  out is a complete
+    NVFP4Tensor afterwards (out.s_dec = 1/s_enc is written by the GEMM), so it
+    can feed the next GEMM directly."""
     s_enc: torch.Tensor           # fp32 [1], read
-    out: NVFP4Tensor              # q [M, N/2], sf tiled; out.s_dec is not written
+    out: NVFP4Tensor              # q [M, N/2], sf tiled, s_dec written
     amax: torch.Tensor | None     # fp32 [1], written with max|Y|
+    activation: int = ACT_NONE    # ACT_GELU: Y = bf16(GELU(alpha * acc))
 
 
 def gemm(a: NVFP4Tensor, b: NVFP4Tensor, y: torch.Tensor | None = None,
@@ -211,7 +219,7 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, y: torch.Tensor | None = None,
     fo = None
     if fused is not None:
         fo = FusedOut(fused.s_enc.data_ptr(), fused.out.q.data_ptr(), fused.out.sf.data_ptr(),
-                      _ptr(fused.amax))
+                      _ptr(fused.amax), fused.out.s_dec.data_ptr(), int(fused.activation))
     _check("nvfp4_gemm", lib().nvfp4_gemm(
         a.q.data_ptr(), a.sf.data_ptr(), a.s_dec.data_ptr(), b.q.data_ptr(), b.sf.data_ptr(),
         b.s_dec.data_ptr(), M, N, K, _ptr(y), ctypes.byref(fo) if fo is not None else None,

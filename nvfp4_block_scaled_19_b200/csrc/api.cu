@@ -194,7 +194,8 @@ nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_
         return NVFP4_ERR_INVALID_ARG;
     if (y_bf16 == nullptr && fused == nullptr) return NVFP4_ERR_INVALID_ARG;
     if (fused != nullptr &&
-        (N % 16 != 0 || fused->s_enc_y == nullptr || fused->yq == nullptr || fused->ysf == nullptr))
+        (N % 16 != 0 || fused->s_enc_y == nullptr || fused->yq == nullptr || fused->ysf == nullptr ||
+         (fused->activation != NVFP4_ACT_NONE && fused->activation != NVFP4_ACT_GELU)))
         return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(aq) || !aligned16(bq) || !aligned16(asf) || !aligned16(bsf) ||
         (y_bf16 != nullptr && !aligned16(y_bf16)))
@@ -224,6 +225,8 @@ nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_
     p.yq = fused ? fused->yq : nullptr;
     p.ysf = fused ? fused->ysf : nullptr;
     p.amax_y = fused ? fused->amax_y : nullptr;
+    p.s_dec_y = fused ? fused->s_dec_y : nullptr;
+    p.act = fused ? fused->activation : NVFP4_ACT_NONE;
     p.M = M;
     p.N = N;
     p.K = K;

@@ -111,7 +111,7 @@ struct GemmConfig {
     static constexpr uint32_t IDESC = make_idesc_mxf4nvf4(kBM, BN);
 };
 
-template <class Cfg>
+template <class Cfg, bool kGelu>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                 const GemmParams p) {
@@ -160,6 +160,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
     float *inv_tab = reinterpret_cast<float *>(smem + Cfg::OFF_INV);
     if (p.yq != nullptr) fill_inv_table(inv_tab, *p.s_enc_y);
+    if (p.s_dec_y != nullptr && blockIdx.x == 0 && threadIdx.x == 0)
+        *p.s_dec_y = __fdiv_rn(1.0f, *p.s_enc_y);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -375,7 +377,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             tc_fence_after();
             // Drain 128 accumulator columns into 64 packed bf16x2 registers.
             uint32_t pk[64];
-            drain_cols<128>(tmem_base + acc * Cfg::BN + col0 + ((static_cast<uint32_t>(quad) * 32) << 16),
+            drain_cols<128, kGelu>(tmem_base + acc * Cfg::BN + col0 + ((static_cast<uint32_t>(quad) * 32) << 16),
                       alpha, pk);
             // Accumulator read: hand it back to the MMA warp.
             tc_fence_before();
@@ -401,14 +403,14 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
 }
 
-template <class Cfg>
+template <class Cfg, bool kGelu>
 static cudaError_t launch_cfg(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
                               int num_sms, cudaStream_t stream) {
     static int configured_device = -1;
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<Cfg>,
+        cudaError_t e = cudaFuncSetAttribute(gemm_kernel<Cfg, kGelu>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return e;
@@ -416,7 +418,7 @@ static cudaError_t launch_cfg(const CUtensorMap &ta, const CUtensorMap &tb, cons
     }
     const int64_t tiles = ((p.M + kBM - 1) / kBM) * ((p.N + Cfg::BN - 1) / Cfg::BN);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-    gemm_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
+    gemm_kernel<Cfg, kGelu><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
     return cudaGetLastError();
 }
 
@@ -437,9 +439,17 @@ namespace nvfp4 {
 
 cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
                         GemmKind kind, int num_sms, cudaStream_t stream) {
-    if (kind == kGemmPair) return launch_pair(ta, tb, p, num_sms, stream);
-    if (kind == kGemm256) return launch_cfg<Cfg256>(ta, tb, p, num_sms, stream);
-    return launch_cfg<Cfg128>(ta, tb, p, num_sms, stream);
+    // The activation is a template parameter, so the plain kernels keep their
+    // register allocation and only the GELU variants carry erff.
+    const bool gelu = p.act == 1;
+    if (kind == kGemmPair)
+        return gelu ? launch_pair<true>(ta, tb, p, num_sms, stream)
+                    : launch_pair<false>(ta, tb, p, num_sms, stream);
+    if (kind == kGemm256)
+        return gelu ? launch_cfg<Cfg256, true>(ta, tb, p, num_sms, stream)
+                    : launch_cfg<Cfg256, false>(ta, tb, p, num_sms, stream);
+    return gelu ? launch_cfg<Cfg128, true>(ta, tb, p, num_sms, stream)
+                : launch_cfg<Cfg128, false>(ta, tb, p, num_sms, stream);
 }
 
 }  // namespace nvfp4

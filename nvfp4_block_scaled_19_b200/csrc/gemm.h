@@ -18,6 +18,8 @@ struct GemmParams {
     uint8_t *yq;            // fused quantize: packed [M, N/2] or null (= no fusion)
     uint8_t *ysf;           // fused quantize: tiled scales
     float *amax_y;          // fused quantize: 1 fp32 (pre-zeroed) or null
+    float *s_dec_y;         // fused quantize: 1 fp32 written with 1/s_enc_y, or null
+    int act;                // 0 none, 1 exact GELU on alpha * acc before the bf16 rounding
     int64_t M, N, K;
     int64_t n_sf_blocks;    // ceil(N / 128): 128-row blocks present in bsf
     int64_t m_sf_blocks;    // ceil(M / 128): 128-row blocks present in asf

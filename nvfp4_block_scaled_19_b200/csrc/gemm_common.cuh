@@ -33,19 +33,48 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n)
     return c;
 }
 
-// Reads NC (64 or 128) fp32 accumulator columns of this warp's 32 TMEM lanes
-// (taddr = lane base + first column), scales by alpha and rounds to packed
-// bf16x2.  Two 32-column loads are in flight at a time.
+// GELU of the fused FFN epilogue, g(h) = 0.5 h (1 + erf(h / sqrt 2)) =
+// 0.5 h erfc(-h / sqrt 2), with erfc(u) for u = |h| / sqrt 2 >= 0 from
+// Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26
+// (Hastings' rational approximation, |error of erf| <= 1.5e-7):
+//   erfc(u) ~ t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-u^2),
+//   t = 1 / (1 + p u).
+// Then g = 0.5 h c for h < 0 (no cancellation) and g = h - 0.5 h c for
+// h >= 0, with c = erfc(u).  The reciprocal and the exponential use the fast
+// hardware approximations; the total error stays far below the bf16
+// rounding of the output, and about half the instructions of erff.
+__device__ __forceinline__ float gelu_erf(float h) {
+    constexpr float p = 0.3275911f, a1 = 0.254829592f, a2 = -0.284496736f,
+                    a3 = 1.421413741f, a4 = -1.453152027f, a5 = 1.061405429f;
+    const float u = fabsf(h) * 0.70710678118654752f;
+    const float t = __fdividef(1.0f, fmaf(p, u, 1.0f));
+    const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, a5, a4), a3), a2), a1);
+    const float c = poly * __expf(-u * u);
+    const float q = 0.5f * h * c;
+    return h >= 0.0f ? h - q : q;
+}
+
+// Scales 32 fp32 accumulator values by alpha, applies the activation (kGelu)
+// and rounds to 16 packed bf16x2.
+template <bool kGelu>
 __device__ __forceinline__ void cvt_32(const uint32_t (&r)[32], float alpha, uint32_t *pk) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
-                                                       __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
+        float h0 = __fmul_rn(__uint_as_float(r[2 * i]), alpha);
+        float h1 = __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha);
+        if (kGelu) {
+            h0 = gelu_erf(h0);
+            h1 = gelu_erf(h1);
+        }
+        const __nv_bfloat162 h = __floats2bfloat162_rn(h0, h1);
         pk[i] = *reinterpret_cast<const uint32_t *>(&h);
     }
 }
 
-template <int NC>
+// Reads NC (64 or 128) fp32 accumulator columns of this warp's 32 TMEM lanes
+// (taddr = lane base + first column) into packed bf16x2 (alpha, activation
+// kGelu, rounding).  Two 32-column loads are in flight at a time.
+template <int NC, bool kGelu>
 __device__ __forceinline__ void drain_cols(uint32_t taddr, float alpha, uint32_t (&pk)[NC / 2]) {
     static_assert(NC == 64 || NC == 128, "64 or 128 columns");
 #pragma unroll
@@ -54,8 +83,8 @@ __device__ __forceinline__ void drain_cols(uint32_t taddr, float alpha, uint32_t
         tmem_ld_32x32b_x32(taddr + ch * 32, r0);
         tmem_ld_32x32b_x32(taddr + ch * 32 + 32, r1);
         tmem_ld_wait();
-        cvt_32(r0, alpha, pk + 16 * ch);
-        cvt_32(r1, alpha, pk + 16 * ch + 16);
+        cvt_32<kGelu>(r0, alpha, pk + 16 * ch);
+        cvt_32<kGelu>(r1, alpha, pk + 16 * ch + 16);
     }
 }
 

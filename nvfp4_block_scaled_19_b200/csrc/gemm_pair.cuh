@@ -74,7 +74,7 @@ struct PairConfig {
     static constexpr uint32_t IDESC = make_idesc_mxf4nvf4(256, 256);
 };
 
-template <class Cfg>
+template <class Cfg, bool kGelu>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_b, const GemmParams p) {
@@ -127,6 +127,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     }
     float *inv_tab = reinterpret_cast<float *>(smem + Cfg::OFF_INV);
     if (p.yq != nullptr) fill_inv_table(inv_tab, *p.s_enc_y);
+    if (p.s_dec_y != nullptr && blockIdx.x == 0 && threadIdx.x == 0)
+        *p.s_dec_y = __fdiv_rn(1.0f, *p.s_enc_y);
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // barrier inits of both CTAs visible before any remote use
@@ -341,12 +343,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
             const TileCoord tc = tile_coord(t, tiles_m, tiles_n);
             if (!mbar_wait_warp(acc_full, local & 1, abort_flag, 16)) break;
             tc_fence_after();
+            const uint32_t taddr = tmem_base + col0 + ((static_cast<uint32_t>(quad) * 32) << 16);
             uint32_t pk[Cfg::EPI_COLS / 2];
-            drain_cols<Cfg::EPI_COLS>(tmem_base + col0 + ((static_cast<uint32_t>(quad) * 32) << 16),
-                                      alpha, pk);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_l);
+            if constexpr (kGelu && Cfg::EPI_COLS == 64) {
+                // All 64 raw columns in registers, accumulator handed back,
+                // then the GELU arithmetic overlaps the next tile's MMAs.
+                uint32_t r0[32], r1[32];
+                tmem_ld_32x32b_x32(taddr, r0);
+                tmem_ld_32x32b_x32(taddr + 32, r1);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_l);
+                cvt_32<true>(r0, alpha, pk);
+                cvt_32<true>(r1, alpha, pk + 16);
+            } else {
+                drain_cols<Cfg::EPI_COLS, kGelu>(taddr, alpha, pk);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_l);
+            }
             store_row<Cfg::EPI_COLS>(p, pk, int64_t(tc.m_blk) * Cfg::BM + row_in_tile,
                           int64_t(tc.n_blk) * Cfg::BN + col0, s_enc_y, inv_tab, amax_bits);
         }
@@ -369,25 +385,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     }
 }
 
-using PairCfg = PairConfig<5, 8>;
+// Plain epilogue: 8 warps of 128 columns.  GELU epilogue: 16 warps of 64
+// columns, so a warp holds its raw columns while it hands the accumulator
+// back and computes the activation afterwards.
+template <bool kGelu>
+using PairCfgFor = PairConfig<5, kGelu ? 16 : 8>;
 
+template <bool kGelu>
 inline cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
                                int num_sms, cudaStream_t stream) {
+    using Cfg = PairCfgFor<kGelu>;
     static int configured[64] = {0};
     static int max_clusters[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!configured[dev]) {
-        e = cudaFuncSetAttribute(gemm_pair_kernel<PairCfg>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM_BYTES);
+        e = cudaFuncSetAttribute(gemm_pair_kernel<Cfg, kGelu>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (num_sms / 2));
-        cfg.blockDim = dim3(PairCfg::THREADS);
-        cfg.dynamicSmemBytes = PairCfg::SMEM_BYTES;
+        cfg.blockDim = dim3(Cfg::THREADS);
+        cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
         int n = 0;
-        e = cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<PairCfg>, &cfg);
+        e = cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<Cfg, kGelu>, &cfg);
         if (e != cudaSuccess || n < 1) {
             cudaGetLastError();
             n = num_sms / 2;
@@ -398,8 +420,8 @@ inline cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
     const int64_t tiles = ((p.M + 255) / 256) * ((p.N + 255) / 256);
     int64_t pairs = max_clusters[dev];
     if (pairs > tiles) pairs = tiles;
-    gemm_pair_kernel<PairCfg><<<static_cast<unsigned>(2 * pairs), PairCfg::THREADS,
-                                PairCfg::SMEM_BYTES, stream>>>(ta, tb, p);
+    gemm_pair_kernel<Cfg, kGelu><<<static_cast<unsigned>(2 * pairs), Cfg::THREADS,
+                                Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
     return cudaGetLastError();
 }
 

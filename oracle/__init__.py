@@ -11,7 +11,8 @@ operands (numpy.matmul), after which nothing is reordered or fused.
 Parity status: every function here is pinned by tests/test_oracle_*.py
 against facts that do not come from the oracle itself (format value sets,
 hand-derived rounding ties, torch's float8_e4m3fn conversion, exact rational
-GEMMs, lossless round trips and the amax-to-6 invariant).
+GEMMs, lossless round trips, the amax-to-6 invariant, and for gelu the
+normal-CDF identities and table values).
 """
 from __future__ import annotations
 
@@ -192,6 +193,19 @@ def gemm_tolerance_ok(gpu: np.ndarray, ref: np.ndarray, rel: float = 1e-2):
         ratio = np.where(bound > 0, err / bound, np.where(err > 0, np.inf, 0.0))
     worst = float(ratio.max()) if ratio.size else 0.0
     return bool(np.all(err <= bound)), worst
+
+
+def gelu(h: np.ndarray) -> np.ndarray:
+    """Exact GELU in fp64, g(h) = h * Phi(h) = 0.5 h (1 + erf(h / sqrt 2)): the
+    activation a fused FFN up-projection epilogue applies before rounding to
+    bf16.  The pages fuse consecutive operations into their GEMM kernels
+    ("NVIDIA показала, как сократить генерацию FLUX 3 Image Klein с 22 до 6
+    секунд", section "Квантование NVFP4 и оптимизация вычислительных ядер")
+    without naming the activation; exact GELU is the reading taken.  One
+    library step: scipy's fp64 erf."""
+    from scipy.special import erf
+    h = np.asarray(h, dtype=np.float64)
+    return 0.5 * h * (1.0 + erf(h / np.sqrt(2.0)))
 
 
 def num_threads() -> int:

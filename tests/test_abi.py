@@ -86,6 +86,9 @@ def test_invalid_arguments_rejected_first(L):
     assert g(p, p, p, p, p, p, 128, 128, 128, p, ctypes.byref(bad), None) == 1
     ok = nv.FusedOut(p, p, p, None)
     assert g(p, p, p, p, p, p, 128, 120, 128, p, ctypes.byref(ok), None) == 1  # N % 16
+    act = nv.FusedOut(p, p, p, None, None, 2)  # no such activation
+    assert g(p, p, p, p, p, p, 128, 128, 128, p, ctypes.byref(act), None) == 1
+    assert ctypes.sizeof(nv.FusedOut) == 48   # five pointers + int, padded (header layout)
     assert L.nvfp4_device_error(None, None) == 1
     qd = L.nvfp4_quantize_dynamic
     assert qd(p, 4, 24, p, p, None, None, p, None) == 1         # cols % 16

@@ -114,6 +114,8 @@ def test_gemm_workloads_sampled_rows(nv, name):
     oracle computes a seeded sample of rows (first, last, random)."""
     w = WORKLOADS[name]
     for li, layer in enumerate(w.layers):
+        if layer.x_from_prev:
+            continue   # fed by the previous layer's fused output: see test_gpu_ffn_fused.py
         x, wt = layer_inputs(w, li)
         M = x.shape[0]
         rng = np.random.default_rng(li)

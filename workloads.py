@@ -36,6 +36,9 @@ class Layer:
     x_dist: str          # "normal_outliers" | "lognormal_channels" | "gelu" | "normal"
     w_std: float | None  # None -> 1/sqrt(K)
     fused_out: bool = False  # output feeds a next-layer NVFP4 quantize
+    act: str = "none"        # activation of a fused epilogue: "none" | "gelu"
+    x_from_prev: bool = False  # X is the previous layer's fused NVFP4 output (not drawn)
+    keep_y: bool = True      # the bf16 Y is needed (False: only the fused output)
 
 
 @dataclass(frozen=True)
@@ -84,6 +87,15 @@ WORKLOADS: dict[str, Workload] = {
                 Layer("attn_out", K=3072, N=3072, x_dist="lognormal_channels", w_std=None),
                 Layer("ffn_up", K=3072, N=12288, x_dist="lognormal_channels", w_std=None),
                 Layer("ffn_down", K=12288, N=3072, x_dist="gelu", w_std=None, fused_out=True))),
+    "ffn_block_2048": Workload(
+        "ffn_block_2048",
+        "DiT FFN block at 2048^2: M=16896; up-projection 3072->12288 whose epilogue applies "
+        "GELU and the NVFP4 quantize, feeding the down-projection 12288->3072 directly",
+        M=16896, seed=5,
+        layers=(Layer("ffn_up", K=3072, N=12288, x_dist="lognormal_channels", w_std=None,
+                      fused_out=True, act="gelu", keep_y=False),
+                Layer("ffn_down", K=12288, N=3072, x_dist="gelu", w_std=None,
+                      x_from_prev=True))),
 }
 
 
@@ -122,11 +134,13 @@ def draw_w(N: int, K: int, std: float | None, seed: int, index: int = 1) -> torc
     return (torch.randn(N, K, generator=g, dtype=torch.float32) * s).to(torch.bfloat16)
 
 
-def layer_inputs(w: Workload, li: int, M: int | None = None) -> tuple[torch.Tensor, torch.Tensor]:
-    """(X, W) for layer li of workload w; M may be overridden (smaller) for tests."""
+def layer_inputs(w: Workload, li: int, M: int | None = None):
+    """(X, W) for layer li of workload w; M may be overridden (smaller) for
+    tests.  X is None for a layer whose input is the previous layer's fused
+    output."""
     l = w.layers[li]
     m = w.M if M is None else M
-    x = draw_x(l.x_dist, m, l.K, w.seed, index=10 * li)
+    x = None if l.x_from_prev else draw_x(l.x_dist, m, l.K, w.seed, index=10 * li)
     wt = draw_w(l.N, l.K, l.w_std, w.seed, index=10 * li + 1)
     return x, wt
 
