@@ -280,6 +280,42 @@ def calibrate(nv, layers) -> None:
     torch.cuda.synchronize()
 
 
+def graph_timing(nv, layers, flush, steps, dist, device, world) -> dict:
+    """The same step captured once in a CUDA graph and replayed (no host
+    launch overhead between the kernels); L2 flushed before every replay,
+    outside the timed span."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        run_step(nv, layers)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            run_step(nv, layers)
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(3):
+        flush.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    barrier(dist, device)
+    for a, b in ev:
+        flush.zero_()
+        a.record()
+        g.replay()
+        b.record()
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    sec = max_over_ranks(ms / 1e3, dist, device)
+    del g
+    flops = sum(L.flops for L in layers) * steps
+    return {"value": round(aggregate(flops, world, sec) / 1e12, 3), "unit": UNIT,
+            "ms_per_step": round(ms / steps, 5), "steps": steps,
+            "kernels_per_step": launches_per_step(layers),
+            "note": "one CUDA graph per step (captured once), events around each replay"}
+
+
 def launches_per_step(layers) -> int:
     return sum(1 + (0 if L.spec.x_from_prev else 1) for L in layers)
 
@@ -350,6 +386,10 @@ def gpu_arm(args) -> dict | None:
     q_gbs = q_bytes / (q_ms_sum * 1e-3) / 1e9 if q_bytes else 0.0
 
     traffic, traffic_src = profiled_traffic(w.name)
+    graph = graph_timing(nv, layers, flush, args.steps, dist, device, world)
+    code, detail = nv.device_error()
+    if code != 0:
+        raise RuntimeError(f"device wait timed out in the graph replays (tag {detail})")
     e2e = host_e2e(nv, layers, args, device, dist, world)
     clocks = sampler.summary()
 
@@ -386,6 +426,7 @@ def gpu_arm(args) -> dict | None:
                      "peak_source": f"{peak_src}: 4 x bf16_tflops burst ({bf16_burst}); "
                                     f"sustained would be {FP4_PER_BF16 * bf16_sust}"},
         "clocks": clocks,
+        "graph": graph,
         "e2e": e2e,
         "gpu_launches": launches_per_step(layers) * args.steps,
     }
