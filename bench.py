@@ -201,14 +201,16 @@ class ClockSampler:
 # ----------------------------------------------------------------- the GPU arm
 
 class Layer:
-    def __init__(self, nv, spec, M, x_cpu, w_cpu, device):
+    def __init__(self, nv, spec, M, x_cpu, w_cpu, device, row_scales=False):
         self.spec = spec
+        self.row_scales = row_scales
         self.M, self.K = M, spec.K
         self.N = w_cpu.shape[0]
         self.x_cpu = x_cpu
         self.x = None if x_cpu is None else x_cpu.to(device)
         self.lin = nv.NVFP4Linear(w_cpu.to(device))
-        self.xq = None if spec.x_from_prev else nv.empty_nvfp4(self.M, self.K, device)
+        self.xq = (None if spec.x_from_prev
+                   else nv.empty_nvfp4(self.M, self.K, device, row_scales=row_scales))
         self.amax = torch.empty(1, dtype=torch.float32, device=device)
         self.y = (torch.empty(self.M, self.N, dtype=torch.bfloat16, device=device)
                   if spec.keep_y else None)
@@ -244,6 +246,8 @@ class Layer:
         if self.spec.x_from_prev:
             return 0
         n = self.M * self.K
+        if self.row_scales:   # one pass over X (the second read of a row hits L1/L2)
+            return 2 * n + n // 2 + nv.sf_bytes(self.M, self.K) + 4 * self.M
         return 2 * n + 2 * n + n // 2 + nv.sf_bytes(self.M, self.K)
 
 
@@ -260,7 +264,11 @@ def run_step(nv, layers, ev=None):
     for i, L in enumerate(layers):
         if ev is not None:
             ev[i][0].record()
-        if not L.spec.x_from_prev:
+        if L.spec.x_from_prev:
+            pass
+        elif L.row_scales:
+            nv.quantize_rowwise(L.x, L.xq)
+        else:
             nv.quantize_dynamic(L.x, L.xq, L.amax)
         if ev is not None:
             ev[i][1].record()
@@ -329,7 +337,9 @@ def gpu_arm(args) -> dict | None:
     nv.lib()
     peaks, peak_src = load_peaks()
     w = WORKLOADS[args.workload]
-    layers = [Layer(nv, l, w.M, *layer_inputs(w, i), device) for i, l in enumerate(w.layers)]
+    row = args.act_scale == "row"
+    layers = [Layer(nv, l, w.M, *layer_inputs(w, i), device, row_scales=row)
+              for i, l in enumerate(w.layers)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     torch.cuda.synchronize()
     calibrate(nv, layers)
@@ -407,14 +417,18 @@ def gpu_arm(args) -> dict | None:
                               + (["input: previous fused output"] if l.x_from_prev else [])
                               for l in w.layers],
                    "l2": "flushed between steps (256 MiB write, outside the timed spans)",
+                   "activation_scale": ("per token (nvfp4_quantize_rowwise, one pass)" if row
+                                        else "per tensor, dynamic (nvfp4_quantize_dynamic)"),
                    "parallelism": f"replicas x{world}"},
         "pct_fp4_peak": {"of_4x_measured_bf16_burst": round(value / world / fp4_peak, 4),
                          "of_nominal_9pf": round(value / world / NOMINAL_FP4_TFLOPS, 4)},
         "quantize": {"gbs": round(q_gbs, 1), "pct_hbm": round(q_gbs / hbm, 4),
                      "ms_per_step": round(q_ms_sum, 5),
-                     "note": "single-launch amax + dynamic quantize of every layer input; "
-                             "algorithmic bytes 4.5625 B/elem + scales (second read from "
-                             "L2 where the input fits)"},
+                     "note": ("per-token quantize, one pass: algorithmic bytes 2.5625 B/elem "
+                              "+ per-row scales" if row else
+                              "single-launch amax + dynamic quantize of every layer input; "
+                              "algorithmic bytes 4.5625 B/elem + scales (second read from "
+                              "L2 where the input fits)")},
         "gemm": {"tflops": round(gemm_tflops, 1), "ms": round(g_avg[top], 5),
                  "layer": layers[top].spec.name},
         "roofline": {"bound": "tensor",
@@ -440,7 +454,7 @@ def host_e2e(nv, layers, args, device, dist, world) -> dict:
     Independent layers go through nvfp4_linear_host; a chain (a layer fed by
     the previous layer's fused output) through the Python API, copying every
     drawn X in and the last layer's Y out."""
-    if any(L.spec.x_from_prev for L in layers):
+    if any(L.spec.x_from_prev or L.row_scales for L in layers):
         return chain_e2e(nv, layers, args, device, dist, world)
     stream = torch.cuda.current_stream()
     hosts = []
@@ -470,16 +484,19 @@ def host_e2e(nv, layers, args, device, dist, world) -> dict:
 
 
 def chain_e2e(nv, layers, args, device, dist, world) -> dict:
+    """End to end through the Python API: every drawn X copied in, every bf16
+    Y the workload produces copied out, pinned host buffers."""
     xs = [(L, L.x_cpu.contiguous().pin_memory()) for L in layers if L.x_cpu is not None]
-    last = layers[-1]
-    yh = torch.empty(last.M, last.N, dtype=torch.bfloat16).pin_memory()
+    ys = [(L, torch.empty(L.M, L.N, dtype=torch.bfloat16).pin_memory())
+          for L in layers if L.y is not None]
     steps = max(1, min(args.steps, args.e2e_steps))
 
     def one():
         for L, xh in xs:
             L.x.copy_(xh, non_blocking=True)
         run_step(nv, layers)
-        yh.copy_(last.y, non_blocking=True)
+        for L, yh in ys:
+            yh.copy_(L.y, non_blocking=True)
 
     for _ in range(2):
         one()
@@ -495,8 +512,8 @@ def chain_e2e(nv, layers, args, device, dist, world) -> dict:
     flops = sum(L.flops for L in layers) * steps
     return {"value": round(aggregate(flops, world, sec) / 1e12, 3), "unit": UNIT,
             "h2d_bytes_per_step": sum(L.M * L.K * 2 for L, _ in xs),
-            "d2h_bytes_per_step": last.M * last.N * 2, "steps": steps,
-            "api": "Python API (quantize_dynamic, gemm with fused epilogue), pinned host buffers"}
+            "d2h_bytes_per_step": sum(L.M * L.N * 2 for L, _ in ys), "steps": steps,
+            "api": "Python API (quantize_dynamic / quantize_rowwise, gemm), pinned host buffers"}
 
 
 # ----------------------------------------------------------------- CPU oracle (baseline / reference)
@@ -595,6 +612,8 @@ def main(argv=None) -> int:
                     help="oracle work timed for cpu_baseline (per reference step: 1/8 of it)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--act-scale", choices=["tensor", "row"], default="tensor",
+                    help="activation tensor scale: per tensor (the pages' scheme) or per token")
     args = ap.parse_args(argv)
     line = reference_arm(args) if args.impl == "reference" else gpu_arm(args)
     if line is not None:

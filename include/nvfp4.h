@@ -198,6 +198,30 @@ nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_
                         int64_t M, int64_t N, int64_t K, void *y_bf16,
                         const nvfp4_fused_out *fused, nvfp4_stream_t stream);
 
+/* Per-token activation scales (the per-tensor FP32 scale of the two-level
+ * scheme taken per row, so an outlier token does not shrink every other
+ * token's block scales).  The pages describe one FP32 scale over the whole
+ * tensor (nmedialink page above, NVFP4 section); this is the finer-grained
+ * variant of that level, with the same per-16 E4M3 block scales.  Row r is
+ * quantized exactly as nvfp4_quantize would quantize the 1-row tensor X[r]
+ * with its own amax (S_enc[r] = 2688 / amax(row r)); the codes and the tiled
+ * scale layout are the usual ones (padding rows get zero scales).
+ *   x_bf16, rows, cols, q_out, sf_out  as for nvfp4_quantize
+ *   s_dec_rows  device, rows fp32, written with 1 / S_enc[r] (4-byte aligned)
+ *   amax_rows   device, rows fp32, written with amax(row r), or NULL
+ * One launch of independent warps (one per row), no grid-wide step. */
+nvfp4_status nvfp4_quantize_rowwise(const void *x_bf16, int64_t rows, int64_t cols,
+                                    uint8_t *q_out, uint8_t *sf_out, float *s_dec_rows,
+                                    float *amax_rows, nvfp4_stream_t stream);
+
+/* nvfp4_gemm with per-row decode scales for A (from nvfp4_quantize_rowwise):
+ * Y[m,n] = bf16(S_dec,A[m] * S_dec,B * sum ...).  a_s_dec_rows holds M fp32
+ * values; everything else as for nvfp4_gemm. */
+nvfp4_status nvfp4_gemm_rowscale(const uint8_t *aq, const uint8_t *asf, const float *a_s_dec_rows,
+                                 const uint8_t *bq, const uint8_t *bsf, const float *b_s_dec,
+                                 int64_t M, int64_t N, int64_t K, void *y_bf16,
+                                 const nvfp4_fused_out *fused, nvfp4_stream_t stream);
+
 /* Device buffers for nvfp4_linear_host (all caller-owned device memory):
  *   x      [M,K] bf16      xq  M*K/2 bytes      xsf  nvfp4_sf_bytes(M,K)
  *   amax   1 fp32          s_dec 1 fp32         y    [M,N] bf16

@@ -80,6 +80,10 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_gemm.restype = st
         L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp,
                                  ctypes.POINTER(FusedOut), vp]
+        L.nvfp4_gemm_rowscale.restype = st
+        L.nvfp4_gemm_rowscale.argtypes = list(L.nvfp4_gemm.argtypes)
+        L.nvfp4_quantize_rowwise.restype = st
+        L.nvfp4_quantize_rowwise.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
         L.nvfp4_linear_host.restype = st
         L.nvfp4_linear_host.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp,
                                         ctypes.POINTER(LinearWorkspace), vp]
@@ -121,16 +125,17 @@ class NVFP4Tensor:
     """A quantized [rows, cols] tensor: packed codes, tiled scales, decode scale."""
     q: torch.Tensor       # uint8 [rows, cols/2]
     sf: torch.Tensor      # uint8 [sf_bytes(rows, cols)]
-    s_dec: torch.Tensor   # float32 [1] = 1 / S_enc
+    s_dec: torch.Tensor   # float32 [1] = 1 / S_enc, or [rows] with per-row scales
     rows: int
     cols: int
 
 
-def empty_nvfp4(rows: int, cols: int, device=None) -> NVFP4Tensor:
+def empty_nvfp4(rows: int, cols: int, device=None, row_scales: bool = False) -> NVFP4Tensor:
     dev = torch.device("cuda") if device is None else device
     return NVFP4Tensor(torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev),
                        torch.empty(sf_bytes(rows, cols), dtype=torch.uint8, device=dev),
-                       torch.empty(1, dtype=torch.float32, device=dev), rows, cols)
+                       torch.empty(rows if row_scales else 1, dtype=torch.float32, device=dev),
+                       rows, cols)
 
 
 def tensor_amax(x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
@@ -196,6 +201,21 @@ def quantize_dynamic(x: torch.Tensor, out: NVFP4Tensor | None = None,
     return out
 
 
+def quantize_rowwise(x: torch.Tensor, out: NVFP4Tensor | None = None,
+                     amax_rows: torch.Tensor | None = None, stream=None) -> NVFP4Tensor:
+    """Per-token activation scales: each row quantized with its own tensor
+    scale 2688 / amax(row); out.s_dec holds one decode scale per row."""
+    _require(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    out = empty_nvfp4(rows, cols, x.device, row_scales=True) if out is None else out
+    if out.s_dec.numel() != rows:
+        raise ValueError("out.s_dec must hold one scale per row")
+    _check("nvfp4_quantize_rowwise", lib().nvfp4_quantize_rowwise(
+        x.data_ptr(), rows, cols, out.q.data_ptr(), out.sf.data_ptr(), out.s_dec.data_ptr(),
+        _ptr(amax_rows), _stream(stream)))
+    return out
+
+
 @dataclass
 class FusedQuant:
     """Fused next-layer quantization outputs of a GEMM.  out is a complete
@@ -220,7 +240,13 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, y: torch.Tensor | None = None,
     if fused is not None:
         fo = FusedOut(fused.s_enc.data_ptr(), fused.out.q.data_ptr(), fused.out.sf.data_ptr(),
                       _ptr(fused.amax), fused.out.s_dec.data_ptr(), int(fused.activation))
-    _check("nvfp4_gemm", lib().nvfp4_gemm(
+    if b.s_dec.numel() != 1:
+        raise ValueError("per-row scales are supported for A (activations) only")
+    row_scaled = a.s_dec.numel() != 1
+    if row_scaled and a.s_dec.numel() != M:
+        raise ValueError("a.s_dec must hold 1 or M decode scales")
+    fn = lib().nvfp4_gemm_rowscale if row_scaled else lib().nvfp4_gemm
+    _check("nvfp4_gemm", fn(
         a.q.data_ptr(), a.sf.data_ptr(), a.s_dec.data_ptr(), b.q.data_ptr(), b.sf.data_ptr(),
         b.s_dec.data_ptr(), M, N, K, _ptr(y), ctypes.byref(fo) if fo is not None else None,
         _stream(stream)))

@@ -182,10 +182,14 @@ nvfp4_status nvfp4_quantize_dynamic(const void *x_bf16, int64_t rows, int64_t co
     return from_cuda(e);
 }
 
-nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_dec,
-                        const uint8_t *bq, const uint8_t *bsf, const float *b_s_dec, int64_t M,
-                        int64_t N, int64_t K, void *y_bf16, const nvfp4_fused_out *fused,
-                        nvfp4_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+nvfp4_status gemm_impl(const uint8_t *aq, const uint8_t *asf, const float *a_s_dec,
+                       const uint8_t *bq, const uint8_t *bsf, const float *b_s_dec, int64_t M,
+                       int64_t N, int64_t K, void *y_bf16, const nvfp4_fused_out *fused,
+                       bool a_row_scale, cudaStream_t stream) {
     if (M < 1 || N < 8 || N % 8 != 0 || K < 64 || K % 64 != 0) return NVFP4_ERR_INVALID_ARG;
     if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31))
         return NVFP4_ERR_INVALID_ARG;
@@ -227,6 +231,7 @@ nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_
     p.amax_y = fused ? fused->amax_y : nullptr;
     p.s_dec_y = fused ? fused->s_dec_y : nullptr;
     p.act = fused ? fused->activation : NVFP4_ACT_NONE;
+    p.a_row_scale = a_row_scale ? 1 : 0;
     p.M = M;
     p.N = N;
     p.K = K;
@@ -237,6 +242,41 @@ nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_
         if (e != cudaSuccess) return NVFP4_ERR_LAUNCH;
     }
     return from_cuda(nvfp4::launch_gemm(ta, tb, p, kind, sms, stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_dec,
+                        const uint8_t *bq, const uint8_t *bsf, const float *b_s_dec, int64_t M,
+                        int64_t N, int64_t K, void *y_bf16, const nvfp4_fused_out *fused,
+                        nvfp4_stream_t stream) {
+    return gemm_impl(aq, asf, a_s_dec, bq, bsf, b_s_dec, M, N, K, y_bf16, fused, false, stream);
+}
+
+nvfp4_status nvfp4_gemm_rowscale(const uint8_t *aq, const uint8_t *asf, const float *a_s_dec_rows,
+                                 const uint8_t *bq, const uint8_t *bsf, const float *b_s_dec,
+                                 int64_t M, int64_t N, int64_t K, void *y_bf16,
+                                 const nvfp4_fused_out *fused, nvfp4_stream_t stream) {
+    return gemm_impl(aq, asf, a_s_dec_rows, bq, bsf, b_s_dec, M, N, K, y_bf16, fused, true,
+                     stream);
+}
+
+nvfp4_status nvfp4_quantize_rowwise(const void *x_bf16, int64_t rows, int64_t cols,
+                                    uint8_t *q_out, uint8_t *sf_out, float *s_dec_rows,
+                                    float *amax_rows, nvfp4_stream_t stream) {
+    nvfp4_status st = check_quantize_args(x_bf16, rows, cols, s_dec_rows, q_out, sf_out);
+    if (st != NVFP4_OK) return st;
+    if ((reinterpret_cast<uintptr_t>(s_dec_rows) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(amax_rows) & 3u) != 0)
+        return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    if (rows == 0) return NVFP4_OK;
+    return from_cuda(nvfp4::launch_quantize_rowwise(x_bf16, rows, cols, q_out, sf_out, s_dec_rows,
+                                                    amax_rows, stream));
 }
 
 nvfp4_status nvfp4_linear_host(const void *x_host_bf16, int64_t M, int64_t K, const uint8_t *wq,

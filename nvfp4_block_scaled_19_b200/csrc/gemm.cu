@@ -365,12 +365,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int quad = warp & 3;        // TMEM lanes [32*quad, 32*quad+32)
         const int col0 = (e >> 2) * 128;  // this warp's 128 columns of the tile
         const int row_in_tile = quad * 32 + lane;
-        const float alpha = __fmul_rn(*p.a_s_dec, *p.b_s_dec);
+        // alpha = S_dec,A * S_dec,B; with per-row scales of A, S_dec,A of this
+        // thread's row of the tile.
+        const float b_s_dec = *p.b_s_dec;
+        const float alpha_tensor = p.a_row_scale ? 0.0f : __fmul_rn(*p.a_s_dec, b_s_dec);
         const float s_enc_y = p.yq != nullptr ? *p.s_enc_y : 1.0f;
         uint32_t amax_bits = 0;
         int local = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
             const TileCoord tc = tile_coord(t, tiles_m, tiles_n);
+            const int64_t m_row = int64_t(tc.m_blk) * kBM + row_in_tile;
+            const float alpha = p.a_row_scale
+                                    ? __fmul_rn(p.a_s_dec[m_row < p.M ? m_row : p.M - 1], b_s_dec)
+                                    : alpha_tensor;
             const int acc = local % Cfg::ACC_STAGES;
             const uint32_t acc_phase = (local / Cfg::ACC_STAGES) & 1;
             if (!mbar_wait_warp(&acc_full[acc], acc_phase, abort_flag, 4)) break;

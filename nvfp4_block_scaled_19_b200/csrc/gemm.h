@@ -20,6 +20,7 @@ struct GemmParams {
     float *amax_y;          // fused quantize: 1 fp32 (pre-zeroed) or null
     float *s_dec_y;         // fused quantize: 1 fp32 written with 1/s_enc_y, or null
     int act;                // 0 none, 1 exact GELU on alpha * acc before the bf16 rounding
+    int a_row_scale;        // 1: a_s_dec holds one decode scale per row of A (per token)
     int64_t M, N, K;
     int64_t n_sf_blocks;    // ceil(N / 128): 128-row blocks present in bsf
     int64_t m_sf_blocks;    // ceil(M / 128): 128-row blocks present in asf
@@ -59,6 +60,10 @@ struct DynWorkspace {
     unsigned pad[3];
 };
 static_assert(sizeof(DynWorkspace) == 32, "workspace size is part of the ABI");
+
+cudaError_t launch_quantize_rowwise(const void *x, int64_t rows, int64_t cols, uint8_t *q,
+                                    uint8_t *sf, float *s_dec_rows, float *amax_rows,
+                                    cudaStream_t stream);
 
 // Returns cudaErrorNotSupported when the rows are too wide for one
 // cooperative grid (then use launch_amax + launch_quantize).

@@ -334,13 +334,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         const int quad = warp & 3;
         const int col0 = (e >> 2) * Cfg::EPI_COLS;
         const int row_in_tile = static_cast<int>(rank) * 128 + quad * 32 + lane;
-        const float alpha = __fmul_rn(*p.a_s_dec, *p.b_s_dec);
+        // alpha = S_dec,A * S_dec,B; with per-row scales of A, S_dec,A of this
+        // thread's row of the tile.
+        const float b_s_dec = *p.b_s_dec;
+        const float alpha_tensor = p.a_row_scale ? 0.0f : __fmul_rn(*p.a_s_dec, b_s_dec);
         const float s_enc_y = p.yq != nullptr ? *p.s_enc_y : 1.0f;
         const uint32_t acc_empty_l = mapa_shared(smem_addr(acc_empty), 0);
         uint32_t amax_bits = 0;
         int local = 0;
         for (int t = pair; t < num_tiles; t += n_pairs, ++local) {
             const TileCoord tc = tile_coord(t, tiles_m, tiles_n);
+            const int64_t m_row = int64_t(tc.m_blk) * Cfg::BM + row_in_tile;
+            const float alpha = p.a_row_scale
+                                    ? __fmul_rn(p.a_s_dec[m_row < p.M ? m_row : p.M - 1], b_s_dec)
+                                    : alpha_tensor;
             if (!mbar_wait_warp(acc_full, local & 1, abort_flag, 16)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + col0 + ((static_cast<uint32_t>(quad) * 32) << 16);

@@ -77,6 +77,23 @@ __device__ __forceinline__ void fill_inv_table(float *tab, float s_enc) {
     }
 }
 
+// Block scale with the multiplier computed directly (for per-row tensor
+// scales, where one table per row would not pay off); same arithmetic as
+// fill_inv_table.
+__device__ __forceinline__ BlockScale block_scale_direct(float a_b, float s_enc) {
+    const float s = __fmul_rn(div6_short(a_b), s_enc);
+    BlockScale b;
+    b.sf = e4m3_encode(s);
+    const float sfv = e4m3_decode(b.sf);
+    float inv = 0.0f;
+    if (sfv != 0.0f) {
+        inv = __fdiv_rn(s_enc, sfv);
+        if (!isfinite(inv)) inv = FLT_MAX;
+    }
+    b.inv = inv;
+    return b;
+}
+
 // Block scale of a 16-element block with amax a_b (a bf16 value):
 //   s = (a_b / 6) * S_enc ; sf = E4M3_rn_satfinite(s) ; inv = tab[sf]
 __device__ __forceinline__ BlockScale block_scale(float a_b, float s_enc, const float *inv_tab) {

@@ -416,6 +416,83 @@ __global__ void __launch_bounds__(kDynThreads) quantize_dynamic_kernel(
                   static_cast<int64_t>(nby) * kStreams, tid % kSliceBlocks, true);
 }
 
+constexpr int kRowWarps = 8;  // rows per CTA of the per-row kernel
+
+// Per-token (per-row) tensor scales: row r is quantized as its own tensor,
+// S_enc[r] = 2688 / amax(row r), with the usual per-16 block scales.  One warp
+// per row: pass 1 reduces the row's amax (lane l takes blocks l, l+32, ...),
+// pass 2 re-reads the row (from L1/L2) and quantizes; four block scales of
+// the row are gathered with shuffles into one 4-byte store.  Warps of the
+// padding rows [rows, pad128(rows)) write zero scale words.  No grid-wide
+// step, so one launch of independent warps.
+__global__ void __launch_bounds__(32 * kRowWarps) quantize_rowwise_kernel(
+    const uint8_t *__restrict__ x, int64_t rows, int64_t cols, uint8_t *__restrict__ q,
+    uint8_t *__restrict__ sf, float *__restrict__ s_dec_rows, float *__restrict__ amax_rows) {
+    const int lane = threadIdx.x & 31;
+    const int64_t r = static_cast<int64_t>(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+    const int64_t kb = cols >> 4;
+    const int64_t kb4 = (kb + 3) >> 2;
+    const int64_t kbp = kb4 << 2;
+    const int64_t rows_pad = (rows + 127) & ~int64_t(127);
+    if (r >= rows_pad) return;
+    if (r >= rows) {
+        for (int64_t c4 = lane; c4 < kb4; c4 += 32)
+            *reinterpret_cast<uint32_t *>(sf + sf_offset(r, 4 * c4, kb4)) = 0u;
+        return;
+    }
+    const uint8_t *xr = x + r * cols * 2;
+    // Pass 1: row amax (16-byte loads that allocate in L1 for pass 2).
+    uint32_t m = 0;
+#pragma unroll 4
+    for (int64_t c = lane; c < kb; c += 32) m = max(m, absmax_bf16x16(ldg_32B(xr + 32 * c, false)));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const float amax = __uint_as_float(m << 16);
+    const float s_enc = tensor_encode_scale(amax);
+    if (lane == 0) {
+        s_dec_rows[r] = __fdiv_rn(1.0f, s_enc);
+        if (amax_rows != nullptr) amax_rows[r] = amax;
+    }
+    // Pass 2: quantize.  All lanes run the same iterations (shuffles).
+    uint8_t *qr = q + r * (cols >> 1);
+    for (int64_t c0 = 0; c0 < kbp; c0 += 32) {
+        const int64_t c = c0 + lane;
+        const bool valid = c < kb;
+        BF16x16 v;
+        if (valid) {
+            v = ldg_32B(xr + 32 * c, false);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v.w[k] = 0u;
+        }
+        const BlockScale bs = block_scale_direct(__uint_as_float(absmax_bf16x16(v) << 16), s_enc);
+        if (valid) {
+            const uint4 lo = make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]);
+            const uint4 hi = make_uint4(v.w[4], v.w[5], v.w[6], v.w[7]);
+            *reinterpret_cast<uint2 *>(qr + 8 * c) =
+                make_uint2(quantize_bf16x8(lo, bs.inv), quantize_bf16x8(hi, bs.inv));
+        }
+        const uint32_t sfc = valid ? bs.sf : 0u;
+        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sfc, 1);
+        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sfc, 2);
+        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sfc, 3);
+        if ((lane & 3) == 0 && c < kbp)
+            *reinterpret_cast<uint32_t *>(sf + sf_offset(r, c, kb4)) =
+                sfc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    }
+}
+
+cudaError_t launch_quantize_rowwise(const void *x, int64_t rows, int64_t cols, uint8_t *q,
+                                    uint8_t *sf, float *s_dec_rows, float *amax_rows,
+                                    cudaStream_t stream) {
+    const int64_t rows_pad = (rows + 127) / 128 * 128;
+    const int64_t blocks = (rows_pad + kRowWarps - 1) / kRowWarps;
+    if (blocks > 2147483647) return cudaErrorInvalidValue;
+    quantize_rowwise_kernel<<<static_cast<unsigned>(blocks), 32 * kRowWarps, 0, stream>>>(
+        reinterpret_cast<const uint8_t *>(x), rows, cols, q, sf, s_dec_rows, amax_rows);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_amax(const void *x, int64_t numel, float *amax, int num_sms,
                         cudaStream_t stream) {
     cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), stream);

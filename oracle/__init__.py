@@ -160,6 +160,45 @@ def dequantize(q: np.ndarray, sf: np.ndarray, s_dec, rows: int, cols: int,
     return out
 
 
+def quantize_rowwise(x_bits: np.ndarray, rows: int, cols: int,
+                     row_idx: np.ndarray | None = None):
+    """Per-token (per-row) tensor scales: row r is quantized exactly as the
+    1-row tensor X[r] with its own dynamic scale (amax, S_enc = 2688/amax,
+    the per-16 block scales of quantize()), its scales placed at row r of the
+    tiled layout.  The pages' per-tensor FP32 scale ("英伟达B200狂飙10.2倍！
+    AI绘图告别龟速！", section "NVFP4量化") taken per row; padding is zero.
+    Returns (q [rows, cols/2], sf tiled, s_dec [rows], amax [rows]); with
+    row_idx only those rows are computed (the others stay zero)."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(rows, cols)
+    kb = cols // 16
+    kbp = (kb + 3) // 4 * 4
+    q = np.zeros((rows, cols // 2), dtype=np.uint8)
+    sf = np.zeros(sf_bytes(rows, cols), dtype=np.uint8)
+    s_dec = np.zeros(rows, dtype=np.float32)
+    amax = np.zeros(rows, dtype=np.float32)
+    for r in (range(rows) if row_idx is None else row_idx):
+        a = tensor_amax(x[r])
+        s_enc = tensor_scale(a)
+        qr, sfr = quantize(x[r], 1, cols, s_enc)
+        q[r] = qr[0]
+        for c in range(kbp):
+            sf[sf_offset(int(r), c, kb)] = sfr[sf_offset(0, c, kb)]
+        s_dec[r] = decode_scale(s_enc)
+        amax[r] = a
+    return q, sf, s_dec, amax
+
+
+def gemm_rowwise(aq, asf, a_sdec_rows, bq, bsf, b_sdec, M: int, N: int, K: int,
+                 rows: np.ndarray | None = None) -> np.ndarray:
+    """ref[m,n] = sum_k x_hat[m,k] w_hat[n,k] in fp64 with per-row decode
+    scales of A: x_hat[m,k] = e2m1 * sf * s_dec[m]."""
+    idx = np.arange(M) if rows is None else np.asarray(rows)
+    a = dequantize(aq, asf, 1.0, M, K, None if rows is None else idx)
+    a = a * np.asarray(a_sdec_rows, dtype=np.float64)[idx][:, None]
+    b = dequantize(bq, bsf, b_sdec, N, K)
+    return np.matmul(a, b.T)
+
+
 # ---------------------------------------------------------------- GEMM
 
 def gemm(aq, asf, a_sdec, bq, bsf, b_sdec, M: int, N: int, K: int,

@@ -32,7 +32,8 @@ def test_header_declares_the_boundary():
     for n in ("nvfp4_tensor_amax", "nvfp4_quantize", "nvfp4_quantize_with_scale", "nvfp4_gemm",
               "nvfp4_packed_bytes", "nvfp4_sf_bytes", "nvfp4_status_string",
               "nvfp4_linear_host", "nvfp4_device_error", "nvfp4_quantize_dynamic",
-              "nvfp4_quantize_dynamic_workspace_bytes"):
+              "nvfp4_quantize_dynamic_workspace_bytes", "nvfp4_quantize_dynamic_noalloc",
+              "nvfp4_quantize_rowwise", "nvfp4_gemm_rowscale"):
         assert n in names
 
 
@@ -95,6 +96,13 @@ def test_invalid_arguments_rejected_first(L):
     assert qd(p, 4, 32, p, p, None, None, None, None) == 1      # no workspace
     assert qd(p, 4, 32, p, p, None, None, p + 4, None) == 2     # misaligned workspace
     assert L.nvfp4_quantize_dynamic_workspace_bytes() == 32
+    qr = L.nvfp4_quantize_rowwise
+    assert qr(p, 4, 24, p, p, p, None, None) == 1              # cols % 16
+    assert qr(p, 4, 32, p, p, None, None, None) == 1           # no per-row scales
+    assert qr(p, 4, 32, p, p, p + 2, None, None) == 2          # misaligned scales
+    gr = L.nvfp4_gemm_rowscale
+    assert gr(p, p, p, p, p, p, 128, 128, 96, p, None, None) == 1     # K % 64
+    assert gr(p, p, p, p, p, p, 128, 128, 128, None, None, None) == 1
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device answer")
