@@ -43,6 +43,7 @@ DEFAULT_WORKLOAD = "qkv_1024"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_PER_BF16 = 4.0      # nominal dense FP4 / dense BF16 (9 / 2.25 PFLOP/s)
+FP8_PER_BF16 = 2.0      # nominal dense FP8 / dense BF16 (4.5 / 2.25 PFLOP/s)
 NOMINAL_FP4_TFLOPS = 9000.0
 
 
@@ -201,16 +202,25 @@ class ClockSampler:
 # ----------------------------------------------------------------- the GPU arm
 
 class Layer:
-    def __init__(self, nv, spec, M, x_cpu, w_cpu, device, row_scales=False):
+    def __init__(self, nv, spec, M, x_cpu, w_cpu, device, row_scales=False, fp8=False):
         self.spec = spec
         self.row_scales = row_scales
+        self.fp8 = fp8
+        if fp8 and spec.x_from_prev:
+            raise ValueError("the FP8 variant takes no NVFP4 fused input")
         self.M, self.K = M, spec.K
         self.N = w_cpu.shape[0]
         self.x_cpu = x_cpu
         self.x = None if x_cpu is None else x_cpu.to(device)
-        self.lin = nv.NVFP4Linear(w_cpu.to(device))
-        self.xq = (None if spec.x_from_prev
-                   else nv.empty_nvfp4(self.M, self.K, device, row_scales=row_scales))
+        if fp8:
+            self.lin = nv.FP8Linear(w_cpu.to(device))
+            self.xq = nv.FP8Tensor(torch.empty(self.M, self.K, dtype=torch.uint8, device=device),
+                                   torch.empty(1, dtype=torch.float32, device=device),
+                                   self.M, self.K)
+        else:
+            self.lin = nv.NVFP4Linear(w_cpu.to(device))
+            self.xq = (None if spec.x_from_prev
+                       else nv.empty_nvfp4(self.M, self.K, device, row_scales=row_scales))
         self.amax = torch.empty(1, dtype=torch.float32, device=device)
         self.y = (torch.empty(self.M, self.N, dtype=torch.bfloat16, device=device)
                   if spec.keep_y else None)
@@ -232,7 +242,11 @@ class Layer:
         """Algorithmic bytes of the GEMM: codes + scales of X and W read once,
         Y (bf16) written once (plus the fused codes + scales when fused)."""
         import nvfp4_block_scaled_19_b200 as nv
-        b = (self.M + self.N) * self.K // 2 + nv.sf_bytes(self.M, self.K) + nv.sf_bytes(self.N, self.K)
+        if self.fp8:
+            b = (self.M + self.N) * self.K
+        else:
+            b = ((self.M + self.N) * self.K // 2 + nv.sf_bytes(self.M, self.K)
+                 + nv.sf_bytes(self.N, self.K))
         b += 2 * self.M * self.N
         if self.fused is not None:
             b += self.M * self.N // 2 + nv.sf_bytes(self.M, self.N)
@@ -246,6 +260,8 @@ class Layer:
         if self.spec.x_from_prev:
             return 0
         n = self.M * self.K
+        if self.fp8:          # amax (read X) + quantize (read X, write 1 B codes)
+            return 2 * n + 2 * n + n
         if self.row_scales:   # one pass over X (the second read of a row hits L1/L2)
             return 2 * n + n // 2 + nv.sf_bytes(self.M, self.K) + 4 * self.M
         return 2 * n + 2 * n + n // 2 + nv.sf_bytes(self.M, self.K)
@@ -266,13 +282,19 @@ def run_step(nv, layers, ev=None):
             ev[i][0].record()
         if L.spec.x_from_prev:
             pass
+        elif L.fp8:
+            nv.tensor_amax(L.x, L.amax)
+            nv.quantize_fp8(L.x, L.amax, L.xq)
         elif L.row_scales:
             nv.quantize_rowwise(L.x, L.xq)
         else:
             nv.quantize_dynamic(L.x, L.xq, L.amax)
         if ev is not None:
             ev[i][1].record()
-        nv.gemm(layer_input(layers, i), L.lin.w, L.y, L.fused, want_y=L.y is not None)
+        if L.fp8:
+            nv.gemm_fp8(L.xq, L.lin.w, L.y, L.fused, want_y=L.y is not None)
+        else:
+            nv.gemm(layer_input(layers, i), L.lin.w, L.y, L.fused, want_y=L.y is not None)
         if ev is not None:
             ev[i][2].record()
 
@@ -325,7 +347,7 @@ def graph_timing(nv, layers, flush, steps, dist, device, world) -> dict:
 
 
 def launches_per_step(layers) -> int:
-    return sum(1 + (0 if L.spec.x_from_prev else 1) for L in layers)
+    return sum(1 + (0 if L.spec.x_from_prev else 2 if L.fp8 else 1) for L in layers)
 
 
 def gpu_arm(args) -> dict | None:
@@ -338,7 +360,8 @@ def gpu_arm(args) -> dict | None:
     peaks, peak_src = load_peaks()
     w = WORKLOADS[args.workload]
     row = args.act_scale == "row"
-    layers = [Layer(nv, l, w.M, *layer_inputs(w, i), device, row_scales=row)
+    fp8 = args.variant == "fp8"
+    layers = [Layer(nv, l, w.M, *layer_inputs(w, i), device, row_scales=row, fp8=fp8)
               for i, l in enumerate(w.layers)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     torch.cuda.synchronize()
@@ -388,14 +411,16 @@ def gpu_arm(args) -> dict | None:
     top = max(range(n_l), key=lambda i: g_avg[i])
     bf16_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     bf16_sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    fp4_peak = FP4_PER_BF16 * bf16_burst
+    per_bf16 = FP8_PER_BF16 if fp8 else FP4_PER_BF16
+    fp4_peak = per_bf16 * bf16_burst
     gemm_tflops = layers[top].flops / (g_avg[top] * 1e-3) / 1e12
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     q_bytes = sum(L.quant_bytes for L in layers)
     q_ms_sum = sum(q_avg[i] for i, L in enumerate(layers) if not L.spec.x_from_prev)
     q_gbs = q_bytes / (q_ms_sum * 1e-3) / 1e9 if q_bytes else 0.0
 
-    traffic, traffic_src = profiled_traffic(w.name)
+    traffic, traffic_src = ((None, "no ncu summary for the FP8 variant") if fp8
+                            else profiled_traffic(w.name))
     graph = graph_timing(nv, layers, flush, args.steps, dist, device, world)
     code, detail = nv.device_error()
     if code != 0:
@@ -410,18 +435,25 @@ def gpu_arm(args) -> dict | None:
         "steps": args.steps, "warmup": max(args.warmup, 3),
         "ms_per_step": round(sum(step_ms) / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "nvfp4 (e2m1 x ue4m3 block scales, fp32 accumulate, bf16 out)",
+        "dtype": ("fp8 (e4m3, per-tensor fp32 scales, fp32 accumulate, bf16 out)" if fp8 else
+                  "nvfp4 (e2m1 x ue4m3 block scales, fp32 accumulate, bf16 out)"),
         "data": "synthetic (seeded DiT-shaped activations and N(0,1/K) weights)",
         "config": {"workload": w.name, "description": w.description, "M": w.M,
                    "layers": [[l.name, l.K, l.N] + (["gelu"] if l.act == "gelu" else [])
                               + (["input: previous fused output"] if l.x_from_prev else [])
                               for l in w.layers],
                    "l2": "flushed between steps (256 MiB write, outside the timed spans)",
+                   "variant": args.variant,
                    "activation_scale": ("per token (nvfp4_quantize_rowwise, one pass)" if row
-                                        else "per tensor, dynamic (nvfp4_quantize_dynamic)"),
+                                        else "per tensor, dynamic (amax + nvfp4_fp8_quantize)"
+                                        if fp8 else
+                                        "per tensor, dynamic (nvfp4_quantize_dynamic)"),
                    "parallelism": f"replicas x{world}"},
         "pct_fp4_peak": {"of_4x_measured_bf16_burst": round(value / world / fp4_peak, 4),
-                         "of_nominal_9pf": round(value / world / NOMINAL_FP4_TFLOPS, 4)},
+                         "of_nominal_9pf": round(value / world / NOMINAL_FP4_TFLOPS, 4)}
+        if not fp8 else
+        {"of_2x_measured_bf16_burst": round(value / world / fp4_peak, 4),
+         "of_nominal_4_5pf": round(value / world / (NOMINAL_FP4_TFLOPS / 2), 4)},
         "quantize": {"gbs": round(q_gbs, 1), "pct_hbm": round(q_gbs / hbm, 4),
                      "ms_per_step": round(q_ms_sum, 5),
                      "note": ("per-token quantize, one pass: algorithmic bytes 2.5625 B/elem "
@@ -432,13 +464,15 @@ def gpu_arm(args) -> dict | None:
         "gemm": {"tflops": round(gemm_tflops, 1), "ms": round(g_avg[top], 5),
                  "layer": layers[top].spec.name},
         "roofline": {"bound": "tensor",
-                     "kernel": gemm_kernel_name(layers[top].M, layers[top].N),
+                     "kernel": ("gemm_pair_kernel FP8 (tcgen05.mma cta_group::2 kind::f8f6f4)"
+                                if fp8 else gemm_kernel_name(layers[top].M, layers[top].N)),
                      "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
                      "traffic": traffic, "traffic_source": traffic_src,
                      "algorithmic_bytes": layers[top].gemm_bytes,
-                     "peak_source": f"{peak_src}: 4 x bf16_tflops burst ({bf16_burst}); "
-                                    f"sustained would be {FP4_PER_BF16 * bf16_sust}"},
+                     "peak_source": f"{peak_src}: {per_bf16:g} x bf16_tflops burst "
+                                    f"({bf16_burst}); sustained would be "
+                                    f"{per_bf16 * bf16_sust}"},
         "clocks": clocks,
         "graph": graph,
         "e2e": e2e,
@@ -454,7 +488,7 @@ def host_e2e(nv, layers, args, device, dist, world) -> dict:
     Independent layers go through nvfp4_linear_host; a chain (a layer fed by
     the previous layer's fused output) through the Python API, copying every
     drawn X in and the last layer's Y out."""
-    if any(L.spec.x_from_prev or L.row_scales for L in layers):
+    if any(L.spec.x_from_prev or L.row_scales or L.fp8 for L in layers):
         return chain_e2e(nv, layers, args, device, dist, world)
     stream = torch.cuda.current_stream()
     hosts = []
@@ -513,7 +547,8 @@ def chain_e2e(nv, layers, args, device, dist, world) -> dict:
     return {"value": round(aggregate(flops, world, sec) / 1e12, 3), "unit": UNIT,
             "h2d_bytes_per_step": sum(L.M * L.K * 2 for L, _ in xs),
             "d2h_bytes_per_step": sum(L.M * L.N * 2 for L, _ in ys), "steps": steps,
-            "api": "Python API (quantize_dynamic / quantize_rowwise, gemm), pinned host buffers"}
+            "api": "Python API (quantize_dynamic / quantize_rowwise / quantize_fp8, gemm), "
+                   "pinned host buffers"}
 
 
 # ----------------------------------------------------------------- CPU oracle (baseline / reference)
@@ -612,6 +647,8 @@ def main(argv=None) -> int:
                     help="oracle work timed for cpu_baseline (per reference step: 1/8 of it)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", choices=["nvfp4", "fp8"], default="nvfp4",
+                    help="nvfp4 (the path) or the FP8 per-tensor variant")
     ap.add_argument("--act-scale", choices=["tensor", "row"], default="tensor",
                     help="activation tensor scale: per tensor (the pages' scheme) or per token")
     args = ap.parse_args(argv)

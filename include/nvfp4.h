@@ -222,6 +222,28 @@ nvfp4_status nvfp4_gemm_rowscale(const uint8_t *aq, const uint8_t *asf, const fl
                                  int64_t M, int64_t N, int64_t K, void *y_bf16,
                                  const nvfp4_fused_out *fused, nvfp4_stream_t stream);
 
+/* FP8 variant: the pages also run the DiT with an FP8 mode ("--variant
+ * fp8r", xalabuda page, section "2. Запуск генерации изображения") without
+ * describing its scaling; read here as E4M3 elements with one FP32 scale per
+ * tensor: S_enc = 448 / amax (1 if amax == 0, FLT_MAX if not finite),
+ * q = E4M3_rn_satfinite(x * S_enc) with the sign kept, S_dec = 1 / S_enc.
+ *   x_bf16      device, [rows, cols] bf16 row-major, cols % 16 == 0
+ *   amax_dev    device, 1 fp32, read (nvfp4_tensor_amax of x, or a static one)
+ *   q_out       device, rows * cols bytes, written (E4M3 codes, row-major)
+ *   s_dec_out   device, 1 fp32, written with 1 / S_enc */
+nvfp4_status nvfp4_fp8_quantize(const void *x_bf16, int64_t rows, int64_t cols,
+                                const float *amax_dev, uint8_t *q_out, float *s_dec_out,
+                                nvfp4_stream_t stream);
+
+/* FP8 GEMM on tcgen05 tensor cores (kind::f8f6f4, CTA pairs), Y = X . W^T
+ * with Y[m,n] = bf16(S_dec,A * S_dec,B * sum_k e4m3(A[m,k]) e4m3(B[n,k])),
+ * fp32 accumulation.  A [M,K] and B [N,K] E4M3 codes from nvfp4_fp8_quantize;
+ * M > 128, N >= 256 with N % 8 == 0, K >= 32 with K % 32 == 0 (other shapes:
+ * NVFP4_ERR_INVALID_ARG).  y_bf16 and fused as for nvfp4_gemm. */
+nvfp4_status nvfp4_fp8_gemm(const uint8_t *a8, const float *a_s_dec, const uint8_t *b8,
+                            const float *b_s_dec, int64_t M, int64_t N, int64_t K, void *y_bf16,
+                            const nvfp4_fused_out *fused, nvfp4_stream_t stream);
+
 /* Device buffers for nvfp4_linear_host (all caller-owned device memory):
  *   x      [M,K] bf16      xq  M*K/2 bytes      xsf  nvfp4_sf_bytes(M,K)
  *   amax   1 fp32          s_dec 1 fp32         y    [M,N] bf16

@@ -84,6 +84,10 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_gemm_rowscale.argtypes = list(L.nvfp4_gemm.argtypes)
         L.nvfp4_quantize_rowwise.restype = st
         L.nvfp4_quantize_rowwise.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
+        L.nvfp4_fp8_quantize.restype = st
+        L.nvfp4_fp8_quantize.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+        L.nvfp4_fp8_gemm.restype = st
+        L.nvfp4_fp8_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
         L.nvfp4_linear_host.restype = st
         L.nvfp4_linear_host.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp,
                                         ctypes.POINTER(LinearWorkspace), vp]
@@ -251,6 +255,64 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, y: torch.Tensor | None = None,
         b.s_dec.data_ptr(), M, N, K, _ptr(y), ctypes.byref(fo) if fo is not None else None,
         _stream(stream)))
     return y
+
+
+@dataclass
+class FP8Tensor:
+    """The FP8 variant's quantized [rows, cols] tensor: E4M3 codes and one
+    decode scale."""
+    q: torch.Tensor       # uint8 [rows, cols]
+    s_dec: torch.Tensor   # float32 [1] = 1 / S_enc = amax / 448
+    rows: int
+    cols: int
+
+
+def quantize_fp8(x: torch.Tensor, amax: torch.Tensor | None = None,
+                 out: FP8Tensor | None = None, stream=None) -> FP8Tensor:
+    """FP8 (E4M3) with one FP32 per-tensor scale 448 / amax; amax computed
+    here (dynamic) unless given (static)."""
+    _require(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    amax = tensor_amax(x, stream=stream) if amax is None else amax
+    if out is None:
+        out = FP8Tensor(torch.empty(rows, cols, dtype=torch.uint8, device=x.device),
+                        torch.empty(1, dtype=torch.float32, device=x.device), rows, cols)
+    _check("nvfp4_fp8_quantize", lib().nvfp4_fp8_quantize(
+        x.data_ptr(), rows, cols, amax.data_ptr(), out.q.data_ptr(), out.s_dec.data_ptr(),
+        _stream(stream)))
+    return out
+
+
+def gemm_fp8(a: FP8Tensor, b: FP8Tensor, y: torch.Tensor | None = None,
+             fused: FusedQuant | None = None, want_y: bool = True, stream=None):
+    """Y[M,N] = A[M,K] . B[N,K]^T on tcgen05 FP8 (E4M3) tensor cores."""
+    M, K, N = a.rows, a.cols, b.rows
+    if b.cols != K:
+        raise ValueError("K mismatch")
+    if y is None and want_y:
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=a.q.device)
+    fo = None
+    if fused is not None:
+        fo = FusedOut(fused.s_enc.data_ptr(), fused.out.q.data_ptr(), fused.out.sf.data_ptr(),
+                      _ptr(fused.amax), fused.out.s_dec.data_ptr(), int(fused.activation))
+    _check("nvfp4_fp8_gemm", lib().nvfp4_fp8_gemm(
+        a.q.data_ptr(), a.s_dec.data_ptr(), b.q.data_ptr(), b.s_dec.data_ptr(), M, N, K, _ptr(y),
+        ctypes.byref(fo) if fo is not None else None, _stream(stream)))
+    return y
+
+
+class FP8Linear:
+    """nn.Linear-shaped FP8 variant: weights quantized once (static scale),
+    activations with a dynamic per-tensor scale on every call."""
+
+    def __init__(self, weight: torch.Tensor):
+        _require(weight, torch.bfloat16, "weight")
+        self.N, self.K = weight.shape
+        self.w = quantize_fp8(weight)
+
+    def __call__(self, x: torch.Tensor, y: torch.Tensor | None = None,
+                 fused: FusedQuant | None = None, want_y: bool = True):
+        return gemm_fp8(quantize_fp8(x), self.w, y, fused, want_y)
 
 
 class NVFP4Linear:

@@ -189,19 +189,21 @@ namespace {
 nvfp4_status gemm_impl(const uint8_t *aq, const uint8_t *asf, const float *a_s_dec,
                        const uint8_t *bq, const uint8_t *bsf, const float *b_s_dec, int64_t M,
                        int64_t N, int64_t K, void *y_bf16, const nvfp4_fused_out *fused,
-                       bool a_row_scale, cudaStream_t stream) {
-    if (M < 1 || N < 8 || N % 8 != 0 || K < 64 || K % 64 != 0) return NVFP4_ERR_INVALID_ARG;
+                       bool a_row_scale, bool fp8, cudaStream_t stream) {
+    if (M < 1 || N < 8 || N % 8 != 0) return NVFP4_ERR_INVALID_ARG;
+    if (fp8 ? (K < 32 || K % 32 != 0 || M <= 128 || N < 256) : (K < 64 || K % 64 != 0))
+        return NVFP4_ERR_INVALID_ARG;
     if (M > (int64_t(1) << 31) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31))
         return NVFP4_ERR_INVALID_ARG;
-    if (aq == nullptr || asf == nullptr || a_s_dec == nullptr || bq == nullptr ||
-        bsf == nullptr || b_s_dec == nullptr)
+    if (aq == nullptr || a_s_dec == nullptr || bq == nullptr || b_s_dec == nullptr ||
+        (!fp8 && (asf == nullptr || bsf == nullptr)))
         return NVFP4_ERR_INVALID_ARG;
     if (y_bf16 == nullptr && fused == nullptr) return NVFP4_ERR_INVALID_ARG;
     if (fused != nullptr &&
         (N % 16 != 0 || fused->s_enc_y == nullptr || fused->yq == nullptr || fused->ysf == nullptr ||
          (fused->activation != NVFP4_ACT_NONE && fused->activation != NVFP4_ACT_GELU)))
         return NVFP4_ERR_INVALID_ARG;
-    if (!aligned16(aq) || !aligned16(bq) || !aligned16(asf) || !aligned16(bsf) ||
+    if (!aligned16(aq) || !aligned16(bq) || (!fp8 && (!aligned16(asf) || !aligned16(bsf))) ||
         (y_bf16 != nullptr && !aligned16(y_bf16)))
         return NVFP4_ERR_MISALIGNED;
     if (fused != nullptr && (!aligned16(fused->yq) || !aligned16(fused->ysf)))
@@ -214,8 +216,9 @@ nvfp4_status gemm_impl(const uint8_t *aq, const uint8_t *asf, const float *a_s_d
     CUtensorMap ta, tb;
     std::memset(&ta, 0, sizeof(ta));
     std::memset(&tb, 0, sizeof(tb));
-    if (!encode_operand_map(&ta, aq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(M), 128) ||
-        !encode_operand_map(&tb, bq, static_cast<uint64_t>(K / 2), static_cast<uint64_t>(N),
+    const uint64_t row_bytes = static_cast<uint64_t>(fp8 ? K : K / 2);
+    if (!encode_operand_map(&ta, aq, row_bytes, static_cast<uint64_t>(M), 128) ||
+        !encode_operand_map(&tb, bq, row_bytes, static_cast<uint64_t>(N),
                             nvfp4::gemm_b_box_rows(kind)))
         return NVFP4_ERR_LAUNCH;
 
@@ -232,6 +235,7 @@ nvfp4_status gemm_impl(const uint8_t *aq, const uint8_t *asf, const float *a_s_d
     p.s_dec_y = fused ? fused->s_dec_y : nullptr;
     p.act = fused ? fused->activation : NVFP4_ACT_NONE;
     p.a_row_scale = a_row_scale ? 1 : 0;
+    p.fp8 = fp8 ? 1 : 0;
     p.M = M;
     p.N = N;
     p.K = K;
@@ -252,7 +256,8 @@ nvfp4_status nvfp4_gemm(const uint8_t *aq, const uint8_t *asf, const float *a_s_
                         const uint8_t *bq, const uint8_t *bsf, const float *b_s_dec, int64_t M,
                         int64_t N, int64_t K, void *y_bf16, const nvfp4_fused_out *fused,
                         nvfp4_stream_t stream) {
-    return gemm_impl(aq, asf, a_s_dec, bq, bsf, b_s_dec, M, N, K, y_bf16, fused, false, stream);
+    return gemm_impl(aq, asf, a_s_dec, bq, bsf, b_s_dec, M, N, K, y_bf16, fused, false, false,
+                     stream);
 }
 
 nvfp4_status nvfp4_gemm_rowscale(const uint8_t *aq, const uint8_t *asf, const float *a_s_dec_rows,
@@ -260,7 +265,32 @@ nvfp4_status nvfp4_gemm_rowscale(const uint8_t *aq, const uint8_t *asf, const fl
                                  int64_t M, int64_t N, int64_t K, void *y_bf16,
                                  const nvfp4_fused_out *fused, nvfp4_stream_t stream) {
     return gemm_impl(aq, asf, a_s_dec_rows, bq, bsf, b_s_dec, M, N, K, y_bf16, fused, true,
-                     stream);
+                     false, stream);
+}
+
+nvfp4_status nvfp4_fp8_quantize(const void *x_bf16, int64_t rows, int64_t cols,
+                                const float *amax_dev, uint8_t *q_out, float *s_dec_out,
+                                nvfp4_stream_t stream) {
+    if (rows < 0 || cols <= 0 || cols % 16 != 0 || rows > (int64_t(1) << 40) / cols)
+        return NVFP4_ERR_INVALID_ARG;
+    if (x_bf16 == nullptr || amax_dev == nullptr || q_out == nullptr || s_dec_out == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(q_out) ||
+        (reinterpret_cast<uintptr_t>(amax_dev) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(s_dec_out) & 3u) != 0)
+        return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    nvfp4_status st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(
+        nvfp4::launch_quantize_fp8(x_bf16, rows * cols, amax_dev, q_out, s_dec_out, sms, stream));
+}
+
+nvfp4_status nvfp4_fp8_gemm(const uint8_t *a8, const float *a_s_dec, const uint8_t *b8,
+                            const float *b_s_dec, int64_t M, int64_t N, int64_t K, void *y_bf16,
+                            const nvfp4_fused_out *fused, nvfp4_stream_t stream) {
+    return gemm_impl(a8, nullptr, a_s_dec, b8, nullptr, b_s_dec, M, N, K, y_bf16, fused, false,
+                     true, stream);
 }
 
 nvfp4_status nvfp4_quantize_rowwise(const void *x_bf16, int64_t rows, int64_t cols,

@@ -21,6 +21,7 @@ struct GemmParams {
     float *s_dec_y;         // fused quantize: 1 fp32 written with 1/s_enc_y, or null
     int act;                // 0 none, 1 exact GELU on alpha * acc before the bf16 rounding
     int a_row_scale;        // 1: a_s_dec holds one decode scale per row of A (per token)
+    int fp8;                // 1: A and B are E4M3 with per-tensor scales only (no asf/bsf)
     int64_t M, N, K;
     int64_t n_sf_blocks;    // ceil(N / 128): 128-row blocks present in bsf
     int64_t m_sf_blocks;    // ceil(M / 128): 128-row blocks present in asf
@@ -60,6 +61,11 @@ struct DynWorkspace {
     unsigned pad[3];
 };
 static_assert(sizeof(DynWorkspace) == 32, "workspace size is part of the ABI");
+
+// FP8 variant: q = E4M3_rn_satfinite(x * 448 / amax), s_dec = amax / 448 (as
+// 1 / S_enc), from a device amax.
+cudaError_t launch_quantize_fp8(const void *x, int64_t numel, const float *amax, uint8_t *q,
+                                float *s_dec_out, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_quantize_rowwise(const void *x, int64_t rows, int64_t cols, uint8_t *q,
                                     uint8_t *sf, float *s_dec_rows, float *amax_rows,

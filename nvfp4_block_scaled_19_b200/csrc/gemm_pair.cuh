@@ -74,7 +74,11 @@ struct PairConfig {
     static constexpr uint32_t IDESC = make_idesc_mxf4nvf4(256, 256);
 };
 
-template <class Cfg, bool kGelu>
+// kFp8: the FP8 variant (E4M3 operands, per-tensor scales only): a 128-byte
+// k-stage holds 128 elements, four tcgen05.mma kind::f8f6f4 (K = 32) cover
+// it, and there are no block scales (no scale copies; the scale warps only
+// forward their arrival so the barrier counts stay the same).
+template <class Cfg, bool kGelu, bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_b, const GemmParams p) {
@@ -100,7 +104,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     const int num_tiles = tiles_m * tiles_n;
     const int pair = blockIdx.x >> 1;
     const int n_pairs = gridDim.x >> 1;
-    const int k_stages = static_cast<int>((p.K + kBK - 1) / kBK);
+    // Operand bytes per row and k-stages of 128 bytes (256 FP4 / 128 FP8
+    // elements); one MMA covers 32 bytes of K.
+    const int64_t kbytes = kFp8 ? p.K : p.K / 2;
+    const int k_stages = static_cast<int>((kbytes + kBKBytes - 1) / kBKBytes);
     const int64_t kb4 = p.K / 64;
 
     if (threadIdx.x == 0) {
@@ -156,27 +163,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                         ok = false;
                         break;
                     }
-                    const int nsub = min(4, static_cast<int>((p.K - int64_t(ks) * kBK) / 64));
+                    const int nsub =
+                        min(4, static_cast<int>((kbytes - int64_t(ks) * kBKBytes) / 32));
                     if (leader)
                         mbar_arrive_expect_tx(&full[stage], 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
-                    uint32_t sf_bytes = sfa_ok ? nsub * 512 : 0;
+                    uint32_t sf_bytes = (!kFp8 && sfa_ok) ? nsub * 512 : 0;
 #pragma unroll
                     for (int rb = 0; rb < 2; ++rb)
-                        if (int64_t(tc.n_blk) * 2 + rb < p.n_sf_blocks) sf_bytes += nsub * 512;
+                        if (!kFp8 && int64_t(tc.n_blk) * 2 + rb < p.n_sf_blocks)
+                            sf_bytes += nsub * 512;
                     mbar_arrive_expect_tx(&sfload[stage], sf_bytes);
                     const uint32_t full_l = full0 + stage * 8;
                     tma_load_2d_pair(&tmap_a, full_l, smem + Cfg::OFF_A + stage * Cfg::A_BYTES,
                                      ks * kBKBytes, a_row, pol_a);
                     tma_load_2d_pair(&tmap_b, full_l, smem + Cfg::OFF_B + stage * Cfg::B_BYTES,
                                      ks * kBKBytes, b_row, pol_b);
-                    if (sfa_ok)
+                    if (!kFp8 && sfa_ok)
                         bulk_load(smem + Cfg::OFF_SFA + stage * Cfg::SFA_BYTES,
                                   p.asf + (sfa_blk * kb4 + int64_t(ks) * 4) * 512, nsub * 512,
                                   &sfload[stage], pol_a);
 #pragma unroll
                     for (int rb = 0; rb < 2; ++rb) {
                         const int64_t brow = int64_t(tc.n_blk) * 2 + rb;
-                        if (brow < p.n_sf_blocks)
+                        if (!kFp8 && brow < p.n_sf_blocks)
                             bulk_load(smem + Cfg::OFF_SFB + stage * Cfg::SFB_BYTES + rb * 2048,
                                       p.bsf + (brow * kb4 + int64_t(ks) * 4) * 512, nsub * 512,
                                       &sfload[stage], pol_b);
@@ -210,8 +219,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         if (leader && lane == 0) {
             const uint64_t adesc0 = make_smem_desc(smem_addr(smem + Cfg::OFF_A), 16, 1024, 2);
             const uint64_t bdesc0 = make_smem_desc(smem_addr(smem + Cfg::OFF_B), 16, 1024, 2);
-            const int k_full = static_cast<int>(p.K / kBK);          // stages of 4 MMAs
-            const int k_tail = static_cast<int>((p.K % kBK) / 64);  // MMAs in a last short stage
+            const int k_full = static_cast<int>(kbytes / kBKBytes);         // stages of 4 MMAs
+            const int k_tail = static_cast<int>((kbytes % kBKBytes) / 32);  // MMAs in a short stage
+            constexpr uint32_t kIdesc = kFp8 ? make_idesc_f8_e4m3(256, 256) : Cfg::IDESC;
+            // One MMA of the stage at smem descriptors (a, b), 32-byte K step j.
+            auto mma = [&](uint64_t a, uint64_t b, uint32_t sfa_t, uint32_t sfb_t, int j,
+                           uint32_t acc) {
+                if constexpr (kFp8)
+                    mma_f8f6f4_pair(tmem_base, a + 2 * j, b + 2 * j, kIdesc, acc);
+                else
+                    mma_mxf4nvf4_pair(tmem_base, a + 2 * j, b + 2 * j, kIdesc, sfa_t + 4 * j,
+                                      sfb_t + 8 * j, acc);
+            };
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -233,12 +252,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                     const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((stage * Cfg::B_BYTES) >> 4);
                     const uint32_t sfa_t = tmem_base + Cfg::SF_BASE + stage * Cfg::SLOT_COLS;
                     const uint32_t sfb_t = sfa_t + Cfg::SFA_COLS;
-                    mma_mxf4nvf4_pair(tmem_base, adesc, bdesc, Cfg::IDESC, sfa_t, sfb_t,
-                                      ks > 0 ? 1u : 0u);
+                    mma(adesc, bdesc, sfa_t, sfb_t, 0, ks > 0 ? 1u : 0u);
 #pragma unroll
-                    for (int j = 1; j < 4; ++j)
-                        mma_mxf4nvf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, Cfg::IDESC,
-                                          sfa_t + 4 * j, sfb_t + 8 * j, 1u);
+                    for (int j = 1; j < 4; ++j) mma(adesc, bdesc, sfa_t, sfb_t, j, 1u);
                     tc_commit_pair(&empty[stage], 0x3);
                     if (++stage == Cfg::STAGES) {
                         stage = 0;
@@ -258,9 +274,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                         const uint32_t sfa_t = tmem_base + Cfg::SF_BASE + stage * Cfg::SLOT_COLS;
                         const uint32_t sfb_t = sfa_t + Cfg::SFA_COLS;
                         for (int j = 0; j < k_tail; ++j)
-                            mma_mxf4nvf4_pair(tmem_base, adesc + 2 * j, bdesc + 2 * j, Cfg::IDESC,
-                                              sfa_t + 4 * j, sfb_t + 8 * j,
-                                              (k_full > 0 || j > 0) ? 1u : 0u);
+                            mma(adesc, bdesc, sfa_t, sfb_t, j, (k_full > 0 || j > 0) ? 1u : 0u);
                         tc_commit_pair(&empty[stage], 0x3);
                         if (++stage == Cfg::STAGES) {
                             stage = 0;
@@ -289,6 +303,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                     ok = false;
                     break;
                 }
+                if constexpr (!kFp8) {
                 const uint32_t slot = lane_base + Cfg::SF_BASE + stage * Cfg::SLOT_COLS;
                 uint32_t va[16];
 #pragma unroll
@@ -319,6 +334,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                     tmem_st_32x32b_x16(slot + Cfg::SFA_COLS + 16 * h, vb);
                 }
                 tmem_st_wait();
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster_relaxed(full0 + stage * 8);
@@ -398,7 +414,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
 template <bool kGelu>
 using PairCfgFor = PairConfig<5, kGelu ? 16 : 8>;
 
-template <bool kGelu>
+template <bool kGelu, bool kFp8>
 inline cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
                                int num_sms, cudaStream_t stream) {
     using Cfg = PairCfgFor<kGelu>;
@@ -408,7 +424,7 @@ inline cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!configured[dev]) {
-        e = cudaFuncSetAttribute(gemm_pair_kernel<Cfg, kGelu>,
+        e = cudaFuncSetAttribute(gemm_pair_kernel<Cfg, kGelu, kFp8>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
@@ -416,7 +432,7 @@ inline cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
         cfg.blockDim = dim3(Cfg::THREADS);
         cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
         int n = 0;
-        e = cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<Cfg, kGelu>, &cfg);
+        e = cudaOccupancyMaxActiveClusters(&n, gemm_pair_kernel<Cfg, kGelu, kFp8>, &cfg);
         if (e != cudaSuccess || n < 1) {
             cudaGetLastError();
             n = num_sms / 2;
@@ -427,7 +443,7 @@ inline cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
     const int64_t tiles = ((p.M + 255) / 256) * ((p.N + 255) / 256);
     int64_t pairs = max_clusters[dev];
     if (pairs > tiles) pairs = tiles;
-    gemm_pair_kernel<Cfg, kGelu><<<static_cast<unsigned>(2 * pairs), Cfg::THREADS,
+    gemm_pair_kernel<Cfg, kGelu, kFp8><<<static_cast<unsigned>(2 * pairs), Cfg::THREADS,
                                 Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
     return cudaGetLastError();
 }

@@ -309,6 +309,18 @@ __device__ __forceinline__ void mma_mxf4nvf4_pair(uint32_t d_tmem, uint64_t a_de
         : "memory");
 }
 
+// CTA-pair D[tmem] (+)= A[smem] . B[smem]^T with E4M3 operands (8-bit, K = 32
+// per instruction), fp32 accumulation, no block scales.
+__device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // D[tmem] (+)= A[smem] . B[smem]^T with E2M1 operands, UE4M3 scales per 16
 // elements (4 per row per K=64 step) read from tensor memory.
 __device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -401,6 +413,14 @@ __device__ __forceinline__ uint64_t make_smem_desc(uint32_t saddr, uint32_t lbo_
 // for .kind::mxf8f6f4/.mxf4/.mxf4nvf4"): A and B E2M1 (format 1) K-major,
 // dense, UE4M3 scales (bit 23 = 0), N>>3 at bits 17-22, M>>4 at bits 24-28,
 // scale-factor ids 0, K = 64.
+// Instruction descriptor of kind::f8f6f4: fp32 accumulator (bits 4-5 = 1),
+// A and B E4M3 (format 0 in bits 7-9 and 10-12), both K-major, N >> 3 at bit
+// 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t make_idesc_f8_e4m3(int M, int N) {
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 __host__ __device__ constexpr uint32_t make_idesc_mxf4nvf4(int M, int N) {
     return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);

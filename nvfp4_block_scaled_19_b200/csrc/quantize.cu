@@ -493,6 +493,55 @@ cudaError_t launch_quantize_rowwise(const void *x, int64_t rows, int64_t cols, u
     return cudaGetLastError();
 }
 
+// FP8 variant (E4M3 elements, one FP32 per-tensor scale, the pages' FP8 mode):
+// S_enc = 448 / amax (1 if amax == 0, FLT_MAX if not finite), each element
+// E4M3_rn_satfinite(x * S_enc) with its sign.  Grid-stride over groups of 8
+// elements: one 16-byte load, four cvt.rn.satfinite.e4m3x2, one 8-byte store.
+__global__ void __launch_bounds__(256) quantize_fp8_kernel(const uint4 *__restrict__ x,
+                                                            int64_t n8, const float *__restrict__ amax,
+                                                            uint2 *__restrict__ q,
+                                                            float *__restrict__ s_dec_out) {
+    const float a = *amax;
+    float s_enc = 1.0f;
+    if (a != 0.0f) {
+        s_enc = __fdiv_rn(448.0f, a);
+        if (!isfinite(s_enc)) s_enc = FLT_MAX;
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0 && s_dec_out != nullptr)
+        *s_dec_out = __fdiv_rn(1.0f, s_enc);
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+         i += stride) {
+        const uint4 v = __ldg(x + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t h[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float lo = __fmul_rn(bf16_lo(w[k]), s_enc);
+            const float hi = __fmul_rn(bf16_hi(w[k]), s_enc);
+            // cvt ... e4m3x2 d, a, b puts a in the upper byte: element 2k+1.
+            asm("{\n\t.reg .b16 t;\n\t"
+                "cvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\t"
+                "cvt.u32.u16 %0, t;\n\t}\n"
+                : "=r"(h[k])
+                : "f"(hi), "f"(lo));
+        }
+        q[i] = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+    }
+}
+
+cudaError_t launch_quantize_fp8(const void *x, int64_t numel, const float *amax, uint8_t *q,
+                                float *s_dec_out, int num_sms, cudaStream_t stream) {
+    const int64_t n8 = numel / 8;
+    int64_t blocks = (n8 + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    quantize_fp8_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        reinterpret_cast<const uint4 *>(x), n8, amax, reinterpret_cast<uint2 *>(q), s_dec_out);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_amax(const void *x, int64_t numel, float *amax, int num_sms,
                         cudaStream_t stream) {
     cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), stream);

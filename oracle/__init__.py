@@ -54,6 +54,10 @@ def lib():
         L.ref_sf_bytes.argtypes = [i64, i64]
         L.ref_sf_offset.restype = i64
         L.ref_sf_offset.argtypes = [i64, i64, i64]
+        L.ref_fp8_tensor_scale.restype = ctypes.c_float
+        L.ref_fp8_tensor_scale.argtypes = [ctypes.c_float]
+        L.ref_quantize_fp8.restype = None
+        L.ref_quantize_fp8.argtypes = [c_u16p, i64, ctypes.c_float, c_u8p]
         L.ref_quantize.restype = None
         L.ref_quantize.argtypes = [c_u16p, i64, i64, ctypes.c_float, c_u8p, c_u8p]
         L.ref_dequantize.restype = None
@@ -197,6 +201,35 @@ def gemm_rowwise(aq, asf, a_sdec_rows, bq, bsf, b_sdec, M: int, N: int, K: int,
     a = a * np.asarray(a_sdec_rows, dtype=np.float64)[idx][:, None]
     b = dequantize(bq, bsf, b_sdec, N, K)
     return np.matmul(a, b.T)
+
+
+def fp8_tensor_scale(amax) -> np.float32:
+    """FP8 variant: S_enc = 448 / amax (1 if 0, FLT_MAX if not finite)."""
+    return np.float32(lib().ref_fp8_tensor_scale(float(np.float32(amax))))
+
+
+def quantize_fp8(x_bits: np.ndarray, rows: int, cols: int):
+    """FP8 (E4M3) with one dynamic FP32 per-tensor scale: returns
+    (q [rows, cols] E4M3 codes, s_dec, amax); see nvfp4_oracle.c for the
+    pages' passage and the reading taken."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(-1)
+    amax = tensor_amax(x)
+    s_enc = fp8_tensor_scale(amax)
+    q = np.empty(x.size, dtype=np.uint8)
+    lib().ref_quantize_fp8(_ptr(x, ctypes.c_uint16), x.size, float(s_enc), _ptr(q, ctypes.c_uint8))
+    return q.reshape(rows, cols), decode_scale(s_enc), amax
+
+
+def dequantize_fp8(q: np.ndarray, s_dec, rows: np.ndarray | None = None) -> np.ndarray:
+    """fp64 x_hat = e4m3(q) * s_dec (all rows or the listed ones)."""
+    table = np.array([e4m3_value(c) if (c & 0x7F) != 0x7F else np.nan for c in range(256)])
+    qq = np.asarray(q) if rows is None else np.asarray(q)[rows]
+    return table[qq] * np.float64(np.float32(s_dec))
+
+
+def gemm_fp8(aq, a_sdec, bq, b_sdec, rows: np.ndarray | None = None) -> np.ndarray:
+    """ref[m,n] = sum_k x_hat[m,k] w_hat[n,k] in fp64 for the FP8 variant."""
+    return np.matmul(dequantize_fp8(aq, a_sdec, rows), dequantize_fp8(bq, b_sdec).T)
 
 
 # ---------------------------------------------------------------- GEMM

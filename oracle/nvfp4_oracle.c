@@ -236,6 +236,31 @@ void ref_gemm_naive(const double *a, const double *b, int64_t M, int64_t N,
         }
 }
 
+/* ---------------- FP8 (E4M3) variant with one FP32 per-tensor scale ----------------
+ * The pages select an FP8 mode beside NVFP4 ("NVIDIA показала, как
+ * сократить генерацию FLUX 3 Image Klein с 22 до 6 секунд", section "2.
+ * Запуск генерации изображения": --variant fp8r) without describing its
+ * scaling; the reading taken is the plainest one: E4M3 elements with one
+ * FP32 scale per tensor, S_enc = 448 / amax (the E4M3 maximum over the tensor
+ * amax; 1 if amax == 0, FLT_MAX if not finite), q = E4M3_rn_satfinite(x * S_enc)
+ * with the sign kept, S_dec = 1 / S_enc. */
+float ref_fp8_tensor_scale(float amax)
+{
+    if (amax == 0.0f) return 1.0f;
+    float s = 448.0f / amax;
+    if (!isfinite(s)) s = FLT_MAX;
+    return s;
+}
+
+void ref_quantize_fp8(const uint16_t *x, int64_t n, float s_enc, uint8_t *q)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; i++) {
+        float v = bf16_to_float(x[i]) * s_enc;
+        q[i] = ref_e4m3_encode(v);
+    }
+}
+
 int ref_num_threads(void)
 {
 #ifdef _OPENMP
