@@ -244,6 +244,16 @@ nvfp4_status nvfp4_fp8_gemm(const uint8_t *a8, const float *a_s_dec, const uint8
                             const float *b_s_dec, int64_t M, int64_t N, int64_t K, void *y_bf16,
                             const nvfp4_fused_out *fused, nvfp4_stream_t stream);
 
+/* Failure-detection self-test (no counterpart on the pages): launches one
+ * warp that waits, through the same bounded mbarrier wait every kernel of
+ * this library uses, on a barrier that is never completed.  After
+ * timeout_us microseconds (1 .. 2000000) the wait gives up, the kernel
+ * records NVFP4_ERR_TIMEOUT with detail NVFP4_SELFTEST_TAG in the device
+ * error word and returns normally: nvfp4_device_error() then reports it, and
+ * the context stays usable.  Faults, traps and hangs are never used. */
+#define NVFP4_SELFTEST_TAG 90
+nvfp4_status nvfp4_selftest_wait_timeout(int64_t timeout_us, nvfp4_stream_t stream);
+
 /* Device buffers for nvfp4_linear_host (all caller-owned device memory):
  *   x      [M,K] bf16      xq  M*K/2 bytes      xsf  nvfp4_sf_bytes(M,K)
  *   amax   1 fp32          s_dec 1 fp32         y    [M,N] bf16

@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_fp8_quantize.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.nvfp4_fp8_gemm.restype = st
         L.nvfp4_fp8_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp]
+        L.nvfp4_selftest_wait_timeout.restype = st
+        L.nvfp4_selftest_wait_timeout.argtypes = [i64, vp]
         L.nvfp4_linear_host.restype = st
         L.nvfp4_linear_host.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp,
                                         ctypes.POINTER(LinearWorkspace), vp]
@@ -313,6 +315,16 @@ class FP8Linear:
     def __call__(self, x: torch.Tensor, y: torch.Tensor | None = None,
                  fused: FusedQuant | None = None, want_y: bool = True):
         return gemm_fp8(quantize_fp8(x), self.w, y, fused, want_y)
+
+
+SELFTEST_TAG = 90
+
+
+def selftest_wait_timeout(timeout_us: int = 50_000, stream=None) -> None:
+    """Failure-detection self-test: a kernel whose bounded wait can never be
+    satisfied gives up after timeout_us; read the result with device_error()."""
+    _check("nvfp4_selftest_wait_timeout",
+           lib().nvfp4_selftest_wait_timeout(int(timeout_us), _stream(stream)))
 
 
 class NVFP4Linear:

@@ -341,6 +341,15 @@ nvfp4_status nvfp4_linear_host(const void *x_host_bf16, int64_t M, int64_t K, co
     return NVFP4_OK;
 }
 
+nvfp4_status nvfp4_selftest_wait_timeout(int64_t timeout_us, nvfp4_stream_t stream) {
+    if (timeout_us < 1 || timeout_us > 2000000) return NVFP4_ERR_INVALID_ARG;
+    int sms = 0;
+    nvfp4_status st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_selftest_wait_timeout(
+        static_cast<uint64_t>(timeout_us) * 1000u, NVFP4_SELFTEST_TAG, stream));
+}
+
 nvfp4_status nvfp4_device_error(int *code_out, int *detail_out) {
     if (code_out == nullptr) return NVFP4_ERR_INVALID_ARG;
     int sms = 0;

@@ -70,6 +70,31 @@ int *device_error_word() {
     return addr[dev];
 }
 
+// Failure-detection self-test: one warp waits, through the kernels' own
+// bounded mbar_wait, on a barrier that nothing will ever complete (its
+// arrival count is 2 and one thread arrives once).  The wait gives up after
+// timeout_ns, records NVFP4_ERR_TIMEOUT with `tag` in the device error word
+// and the kernel returns normally, so the context stays usable.
+__global__ void selftest_wait_timeout_kernel(uint64_t timeout_ns, int tag) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 2);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_arrive(&bar);   // one of the two arrivals; the phase stays open
+    __syncwarp();
+    if (threadIdx.x == 0) mbar_wait_for(&bar, 0, &abort_flag, tag, timeout_ns);
+    __syncwarp();
+}
+
+cudaError_t launch_selftest_wait_timeout(uint64_t timeout_ns, int tag, cudaStream_t stream) {
+    selftest_wait_timeout_kernel<<<1, 32, 0, stream>>>(timeout_ns, tag);
+    return cudaGetLastError();
+}
+
 constexpr int kBM = 128;
 constexpr int kBKBytes = 128;  // 256 FP4 elements per k-stage per row
 constexpr int kBK = 256;

@@ -62,6 +62,8 @@ struct DynWorkspace {
 };
 static_assert(sizeof(DynWorkspace) == 32, "workspace size is part of the ABI");
 
+cudaError_t launch_selftest_wait_timeout(uint64_t timeout_ns, int tag, cudaStream_t stream);
+
 // FP8 variant: q = E4M3_rn_satfinite(x * 448 / amax), s_dec = amax / 448 (as
 // 1 / S_enc), from a device amax.
 cudaError_t launch_quantize_fp8(const void *x, int64_t numel, const float *amax, uint8_t *q,

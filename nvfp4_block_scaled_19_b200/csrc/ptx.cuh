@@ -74,21 +74,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Waits for the phase with the given parity to complete.  Gives up (and
 // returns false) when *abort is set by another thread of the CTA, or after
-// kWaitTimeoutNs, in which case it records the timeout and sets *abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          int tag) {
+// timeout_ns, in which case it records the timeout and sets *abort.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                              int tag, uint64_t timeout_ns) {
     const uint32_t a = smem_addr(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         if (mbar_try_wait(a, parity)) return true;
         if (*abort) return false;
-        if (globaltimer() - t0 > kWaitTimeoutNs) {
+        if (globaltimer() - t0 > timeout_ns) {
             record_timeout(tag);
             *abort = 1;
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          int tag) {
+    return mbar_wait_for(bar, parity, abort, tag, kWaitTimeoutNs);
 }
 
 // Warp-uniform wait: lane 0 polls, every lane gets the same answer, so a
