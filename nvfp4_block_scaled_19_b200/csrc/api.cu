@@ -83,6 +83,22 @@ bool encode_operand_map(CUtensorMap *m, const void *base, uint64_t row_bytes, ui
     return r == CUDA_SUCCESS;
 }
 
+// 2-D bf16 tensor [rows, cols] (row-major) for TMA stores of 32-row x 64-column
+// boxes (128 bytes per row, 128-byte swizzle); out-of-range rows and columns
+// of a box are not written.
+bool encode_output_map(CUtensorMap *m, void *base, uint64_t cols, uint64_t rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 nvfp4_status check_quantize_args(const void *x, int64_t rows, int64_t cols, const void *scale,
                                  const uint8_t *q, const uint8_t *sf) {
     if (rows < 0 || cols <= 0 || cols % 16 != 0) return NVFP4_ERR_INVALID_ARG;
@@ -221,6 +237,11 @@ nvfp4_status gemm_impl(const uint8_t *aq, const uint8_t *asf, const float *a_s_d
         !encode_operand_map(&tb, bq, row_bytes, static_cast<uint64_t>(N),
                             nvfp4::gemm_b_box_rows(kind)))
         return NVFP4_ERR_LAUNCH;
+    CUtensorMap ty;
+    std::memset(&ty, 0, sizeof(ty));
+    if (y_bf16 != nullptr &&
+        !encode_output_map(&ty, y_bf16, static_cast<uint64_t>(N), static_cast<uint64_t>(M)))
+        return NVFP4_ERR_LAUNCH;
 
     nvfp4::GemmParams p;
     p.asf = asf;
@@ -245,7 +266,7 @@ nvfp4_status gemm_impl(const uint8_t *aq, const uint8_t *asf, const float *a_s_d
         cudaError_t e = cudaMemsetAsync(p.amax_y, 0, sizeof(float), stream);
         if (e != cudaSuccess) return NVFP4_ERR_LAUNCH;
     }
-    return from_cuda(nvfp4::launch_gemm(ta, tb, p, kind, sms, stream));
+    return from_cuda(nvfp4::launch_gemm(ta, tb, ty, p, kind, sms, stream));
 }
 
 }  // namespace

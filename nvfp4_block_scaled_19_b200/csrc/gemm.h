@@ -39,8 +39,8 @@ GemmKind gemm_kind(int64_t M, int64_t N);
 // Rows of the B (weight) TMA box for a kernel variant.
 inline uint32_t gemm_b_box_rows(GemmKind k) { return k == kGemm256 ? 256u : 128u; }
 
-cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
-                        GemmKind kind, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty,
+                        const GemmParams &p, GemmKind kind, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_amax(const void *x, int64_t numel, float *amax, int num_sms,
                         cudaStream_t stream);

@@ -96,9 +96,10 @@ __device__ __forceinline__ void drain_cols(uint32_t taddr, float alpha, uint32_t
 template <int NC>
 __device__ __forceinline__ void store_row(const GemmParams &p, const uint32_t (&pk)[NC / 2],
                                           int64_t m, int64_t n0, float s_enc_y,
-                                          const float *inv_tab, uint32_t &amax_bits) {
+                                          const float *inv_tab, uint32_t &amax_bits,
+                                          bool write_y = true) {
     const bool row_ok = m < p.M;
-    if (row_ok && p.y != nullptr) {
+    if (row_ok && p.y != nullptr && write_y) {
         uint8_t *yrow = p.y + (m * p.N + n0) * 2;
         if (n0 + NC <= p.N && (p.N & 15) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 31) == 0) {
 #pragma unroll
