@@ -99,6 +99,24 @@ bool encode_output_map(CUtensorMap *m, void *base, uint64_t cols, uint64_t rows)
     return r == CUDA_SUCCESS;
 }
 
+// Tiled scale factors of a [rows, K] NVFP4 tensor as a 3-D byte tensor
+// [ceil(rows / 128) blocks][K / 32 lines][256 bytes] (each 512-byte tile of
+// 128 rows x 4 blocks is two lines), for boxes of 8 lines (one 256-element
+// k-stage) x box_blocks row blocks.
+bool encode_sf_map(CUtensorMap *m, const void *base, int64_t rows, int64_t K, uint32_t box_blocks) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    const uint64_t lines = static_cast<uint64_t>(K / 32);
+    cuuint64_t dims[3] = {256, lines, static_cast<uint64_t>((rows + 127) / 128)};
+    cuuint64_t strides[2] = {256, 256 * lines};
+    cuuint32_t box[3] = {256, 8, box_blocks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 nvfp4_status check_quantize_args(const void *x, int64_t rows, int64_t cols, const void *scale,
                                  const uint8_t *q, const uint8_t *sf) {
     if (rows < 0 || cols <= 0 || cols % 16 != 0) return NVFP4_ERR_INVALID_ARG;
@@ -229,18 +247,18 @@ nvfp4_status gemm_impl(const uint8_t *aq, const uint8_t *asf, const float *a_s_d
     if (st != NVFP4_OK) return st;
 
     const nvfp4::GemmKind kind = nvfp4::gemm_kind(M, N);
-    CUtensorMap ta, tb;
-    std::memset(&ta, 0, sizeof(ta));
-    std::memset(&tb, 0, sizeof(tb));
+    nvfp4::GemmMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
     const uint64_t row_bytes = static_cast<uint64_t>(fp8 ? K : K / 2);
-    if (!encode_operand_map(&ta, aq, row_bytes, static_cast<uint64_t>(M), 128) ||
-        !encode_operand_map(&tb, bq, row_bytes, static_cast<uint64_t>(N),
+    if (!encode_operand_map(&maps.a, aq, row_bytes, static_cast<uint64_t>(M), 128) ||
+        !encode_operand_map(&maps.b, bq, row_bytes, static_cast<uint64_t>(N),
                             nvfp4::gemm_b_box_rows(kind)))
         return NVFP4_ERR_LAUNCH;
-    CUtensorMap ty;
-    std::memset(&ty, 0, sizeof(ty));
     if (y_bf16 != nullptr &&
-        !encode_output_map(&ty, y_bf16, static_cast<uint64_t>(N), static_cast<uint64_t>(M)))
+        !encode_output_map(&maps.y, y_bf16, static_cast<uint64_t>(N), static_cast<uint64_t>(M)))
+        return NVFP4_ERR_LAUNCH;
+    if (kind == nvfp4::kGemmPair && !fp8 &&
+        (!encode_sf_map(&maps.sfa, asf, M, K, 1) || !encode_sf_map(&maps.sfb, bsf, N, K, 2)))
         return NVFP4_ERR_LAUNCH;
 
     nvfp4::GemmParams p;
@@ -266,7 +284,7 @@ nvfp4_status gemm_impl(const uint8_t *aq, const uint8_t *asf, const float *a_s_d
         cudaError_t e = cudaMemsetAsync(p.amax_y, 0, sizeof(float), stream);
         if (e != cudaSuccess) return NVFP4_ERR_LAUNCH;
     }
-    return from_cuda(nvfp4::launch_gemm(ta, tb, ty, p, kind, sms, stream));
+    return from_cuda(nvfp4::launch_gemm(maps, p, kind, sms, stream));
 }
 
 }  // namespace

@@ -469,24 +469,24 @@ GemmKind gemm_kind(int64_t M, int64_t N) {
 
 namespace nvfp4 {
 
-cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty,
-                        const GemmParams &p, GemmKind kind, int num_sms, cudaStream_t stream) {
+cudaError_t launch_gemm(const GemmMaps &maps, const GemmParams &p, GemmKind kind, int num_sms,
+                        cudaStream_t stream) {
     // The activation is a template parameter, so the plain kernels keep their
     // register allocation and only the GELU variants carry erff.
     const bool gelu = p.act == 1;
     if (p.fp8) {  // the FP8 variant runs on CTA pairs only (the entry point checks the shape)
         if (kind != kGemmPair) return cudaErrorInvalidValue;
-        return gelu ? launch_pair<true, true>(ta, tb, ty, p, num_sms, stream)
-                    : launch_pair<false, true>(ta, tb, ty, p, num_sms, stream);
+        return gelu ? launch_pair<true, true>(maps, p, num_sms, stream)
+                    : launch_pair<false, true>(maps, p, num_sms, stream);
     }
     if (kind == kGemmPair)
-        return gelu ? launch_pair<true, false>(ta, tb, ty, p, num_sms, stream)
-                    : launch_pair<false, false>(ta, tb, ty, p, num_sms, stream);
+        return gelu ? launch_pair<true, false>(maps, p, num_sms, stream)
+                    : launch_pair<false, false>(maps, p, num_sms, stream);
     if (kind == kGemm256)
-        return gelu ? launch_cfg<Cfg256, true>(ta, tb, p, num_sms, stream)
-                    : launch_cfg<Cfg256, false>(ta, tb, p, num_sms, stream);
-    return gelu ? launch_cfg<Cfg128, true>(ta, tb, p, num_sms, stream)
-                : launch_cfg<Cfg128, false>(ta, tb, p, num_sms, stream);
+        return gelu ? launch_cfg<Cfg256, true>(maps.a, maps.b, p, num_sms, stream)
+                    : launch_cfg<Cfg256, false>(maps.a, maps.b, p, num_sms, stream);
+    return gelu ? launch_cfg<Cfg128, true>(maps.a, maps.b, p, num_sms, stream)
+                : launch_cfg<Cfg128, false>(maps.a, maps.b, p, num_sms, stream);
 }
 
 }  // namespace nvfp4

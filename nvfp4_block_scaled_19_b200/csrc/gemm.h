@@ -39,8 +39,16 @@ GemmKind gemm_kind(int64_t M, int64_t N);
 // Rows of the B (weight) TMA box for a kernel variant.
 inline uint32_t gemm_b_box_rows(GemmKind k) { return k == kGemm256 ? 256u : 128u; }
 
-cudaError_t launch_gemm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty,
-                        const GemmParams &p, GemmKind kind, int num_sms, cudaStream_t stream);
+// Tensor maps of one GEMM launch: A and B codes, Y (bf16, may be unused),
+// and for the CTA-pair kernel the scale factors as 3-D byte tensors
+// [128-row blocks][K / 32 lines][256 bytes] (a 512-byte scale tile is two
+// lines), so one box brings a k-stage's scales of one or two row blocks.
+struct GemmMaps {
+    CUtensorMap a, b, y, sfa, sfb;
+};
+
+cudaError_t launch_gemm(const GemmMaps &maps, const GemmParams &p, GemmKind kind, int num_sms,
+                        cudaStream_t stream);
 
 cudaError_t launch_amax(const void *x, int64_t numel, float *amax, int num_sms,
                         cudaStream_t stream);

@@ -87,9 +87,7 @@ struct PairConfig {
 // forward their arrival so the barrier counts stay the same).
 template <class Cfg, bool kGelu, bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
-    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                     const __grid_constant__ CUtensorMap tmap_b,
-                     const __grid_constant__ CUtensorMap tmap_y, const GemmParams p) {
+    gemm_pair_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -116,7 +114,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
     // elements); one MMA covers 32 bytes of K.
     const int64_t kbytes = kFp8 ? p.K : p.K / 2;
     const int k_stages = static_cast<int>((kbytes + kBKBytes - 1) / kBKBytes);
-    const int64_t kb4 = p.K / 64;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) {
@@ -133,8 +130,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        prefetch_tmap(&tmap_a);
-        prefetch_tmap(&tmap_b);
+        prefetch_tmap(&maps.a);
+        prefetch_tmap(&maps.b);
+        if (!kFp8) {
+            prefetch_tmap(&maps.sfa);
+            prefetch_tmap(&maps.sfb);
+        }
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_holder, Cfg::TMEM_COLS);
@@ -164,42 +165,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                 const TileCoord tc = tile_coord(t, tiles_m, tiles_n);
                 const int a_row = tc.m_blk * Cfg::BM + static_cast<int>(rank) * 128;
                 const int b_row = tc.n_blk * Cfg::BN + static_cast<int>(rank) * 128;
-                const int64_t sfa_blk = int64_t(tc.m_blk) * 2 + rank;
-                const bool sfa_ok = sfa_blk < p.m_sf_blocks;
+                const int sfa_blk = tc.m_blk * 2 + static_cast<int>(rank);
                 for (int ks = 0; ks < k_stages; ++ks) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, 11)) {
                         ok = false;
                         break;
                     }
-                    const int nsub =
-                        min(4, static_cast<int>((kbytes - int64_t(ks) * kBKBytes) / 32));
                     if (leader)
                         mbar_arrive_expect_tx(&full[stage], 2 * (Cfg::A_BYTES + Cfg::B_BYTES));
-                    uint32_t sf_bytes = (!kFp8 && sfa_ok) ? nsub * 512 : 0;
-#pragma unroll
-                    for (int rb = 0; rb < 2; ++rb)
-                        if (!kFp8 && int64_t(tc.n_blk) * 2 + rb < p.n_sf_blocks)
-                            sf_bytes += nsub * 512;
-                    mbar_arrive_expect_tx(&sfload[stage], sf_bytes);
-                    if (!kFp8 && sfa_ok)
-                        bulk_load(smem + Cfg::OFF_SFA + stage * Cfg::SFA_BYTES,
-                                  p.asf + (sfa_blk * kb4 + int64_t(ks) * 4) * 512, nsub * 512,
-                                  &sfload[stage], pol_a);
-#pragma unroll
-                    for (int rb = 0; rb < 2; ++rb) {
-                        const int64_t brow = int64_t(tc.n_blk) * 2 + rb;
-                        if (!kFp8 && brow < p.n_sf_blocks)
-                            bulk_load(smem + Cfg::OFF_SFB + stage * Cfg::SFB_BYTES + rb * 2048,
-                                      p.bsf + (brow * kb4 + int64_t(ks) * 4) * 512, nsub * 512,
-                                      &sfload[stage], pol_b);
+                    // One box per operand's scales: 8 lines (this k-stage's four
+                    // 512-byte tiles) of this CTA's A row block, and of both B row
+                    // blocks of the tile.  Boxes are counted whole; lines past K
+                    // or row blocks past the tensor arrive as zeros.
+                    mbar_arrive_expect_tx(&sfload[stage],
+                                          kFp8 ? 0u : uint32_t(Cfg::SFA_BYTES + Cfg::SFB_BYTES));
+                    if (!kFp8) {
+                        tma_load_3d(&maps.sfa, &sfload[stage],
+                                    smem + Cfg::OFF_SFA + stage * Cfg::SFA_BYTES, 0, ks * 8,
+                                    sfa_blk, pol_a);
+                        tma_load_3d(&maps.sfb, &sfload[stage],
+                                    smem + Cfg::OFF_SFB + stage * Cfg::SFB_BYTES, 0, ks * 8,
+                                    tc.n_blk * 2, pol_b);
                     }
                     // Operands after the scales: the scales travel a longer way
                     // (scale warps, TMEM) before the stage is ready; issued
                     // first they land first (measured 1-4% faster on B200).
                     const uint32_t full_l = full0 + stage * 8;
-                    tma_load_2d_pair(&tmap_a, full_l, smem + Cfg::OFF_A + stage * Cfg::A_BYTES,
+                    tma_load_2d_pair(&maps.a, full_l, smem + Cfg::OFF_A + stage * Cfg::A_BYTES,
                                      ks * kBKBytes, a_row, pol_a);
-                    tma_load_2d_pair(&tmap_b, full_l, smem + Cfg::OFF_B + stage * Cfg::B_BYTES,
+                    tma_load_2d_pair(&maps.b, full_l, smem + Cfg::OFF_B + stage * Cfg::B_BYTES,
                                      ks * kBKBytes, b_row, pol_b);
                     if (issued < Cfg::STAGES) ++issued;
                     if (++stage == Cfg::STAGES) {
@@ -421,7 +415,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                         // A box starting inside Y (partial boxes are clipped by
                         // the TMA); boxes that would start past M or N are skipped.
                         if (lane == 0 && m0 < p.M && n0 + 64 * h < p.N) {
-                            tma_store_2d(&tmap_y, stg, static_cast<int>(n0 + 64 * h),
+                            tma_store_2d(&maps.y, stg, static_cast<int>(n0 + 64 * h),
                                          static_cast<int>(m0));
                             bulk_commit_group();
                         }
@@ -461,9 +455,8 @@ template <bool kGelu>
 using PairCfgFor = PairConfig<5, kGelu ? 16 : 8>;
 
 template <bool kGelu, bool kFp8>
-inline cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &ty,
-                               const GemmParams &p,
-                               int num_sms, cudaStream_t stream) {
+inline cudaError_t launch_pair(const GemmMaps &maps, const GemmParams &p, int num_sms,
+                               cudaStream_t stream) {
     using Cfg = PairCfgFor<kGelu>;
     static int configured[64] = {0};
     static int max_clusters[64] = {0};
@@ -491,7 +484,7 @@ inline cudaError_t launch_pair(const CUtensorMap &ta, const CUtensorMap &tb, con
     int64_t pairs = max_clusters[dev];
     if (pairs > tiles) pairs = tiles;
     gemm_pair_kernel<Cfg, kGelu, kFp8><<<static_cast<unsigned>(2 * pairs), Cfg::THREADS,
-                                Cfg::SMEM_BYTES, stream>>>(ta, tb, ty, p);
+                                Cfg::SMEM_BYTES, stream>>>(maps, p);
     return cudaGetLastError();
 }
 

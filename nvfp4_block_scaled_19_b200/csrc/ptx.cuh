@@ -183,6 +183,17 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *m, uint32_t 
         : "memory");
 }
 
+// 3-D tiled TMA load into this CTA's shared memory, completion on `bar`.
+// No multicast.
+__device__ __forceinline__ void tma_load_3d(const CUtensorMap *m, uint64_t *bar, void *dst, int x,
+                                            int y, int z, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_addr(dst)),
+        "l"(m), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
+        : "memory");
+}
+
 // Contiguous bulk copy global -> shared (16-byte aligned, size % 16 == 0).
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
                                           uint64_t *bar, uint64_t policy) {
