@@ -257,13 +257,11 @@ nvfp4_status gemm_impl(const uint8_t *aq, const uint8_t *asf, const float *a_s_d
     if (y_bf16 != nullptr &&
         !encode_output_map(&maps.y, y_bf16, static_cast<uint64_t>(N), static_cast<uint64_t>(M)))
         return NVFP4_ERR_LAUNCH;
-    if (kind == nvfp4::kGemmPair && !fp8 &&
-        (!encode_sf_map(&maps.sfa, asf, M, K, 1) || !encode_sf_map(&maps.sfb, bsf, N, K, 2)))
+    if (!fp8 && (!encode_sf_map(&maps.sfa, asf, M, K, 1) ||
+                 !encode_sf_map(&maps.sfb, bsf, N, K, kind == nvfp4::kGemm128 ? 1 : 2)))
         return NVFP4_ERR_LAUNCH;
 
     nvfp4::GemmParams p;
-    p.asf = asf;
-    p.bsf = bsf;
     p.a_s_dec = a_s_dec;
     p.b_s_dec = b_s_dec;
     p.y = static_cast<uint8_t *>(y_bf16);
@@ -278,8 +276,6 @@ nvfp4_status gemm_impl(const uint8_t *aq, const uint8_t *asf, const float *a_s_d
     p.M = M;
     p.N = N;
     p.K = K;
-    p.n_sf_blocks = (N + 127) / 128;
-    p.m_sf_blocks = (M + 127) / 128;
     if (p.amax_y != nullptr) {
         cudaError_t e = cudaMemsetAsync(p.amax_y, 0, sizeof(float), stream);
         if (e != cudaSuccess) return NVFP4_ERR_LAUNCH;

@@ -138,8 +138,7 @@ struct GemmConfig {
 
 template <class Cfg, bool kGelu>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                const GemmParams p) {
+    gemm_kernel(const __grid_constant__ GemmMaps maps, const GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -159,7 +158,6 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     const int tiles_n = static_cast<int>((p.N + Cfg::BN - 1) / Cfg::BN);
     const int num_tiles = tiles_m * tiles_n;
     const int k_stages = static_cast<int>((p.K + kBK - 1) / kBK);
-    const int64_t kb4 = p.K / 64;  // scale tiles per 128-row block (K % 64 == 0)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::STAGES; ++s) {
@@ -176,8 +174,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        prefetch_tmap(&tmap_a);
-        prefetch_tmap(&tmap_b);
+        prefetch_tmap(&maps.a);
+        prefetch_tmap(&maps.b);
+        prefetch_tmap(&maps.sfa);
+        prefetch_tmap(&maps.sfb);
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, Cfg::TMEM_COLS);
@@ -203,33 +203,25 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
                 const TileCoord tc = tile_coord(t, tiles_m, tiles_n);
-                const uint8_t *asf = p.asf + int64_t(tc.m_blk) * kb4 * 512;
                 for (int ks = 0; ks < k_stages; ++ks) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, 1)) {
                         ok = false;
                         break;
                     }
-                    const int nsub = min(4, static_cast<int>((p.K - int64_t(ks) * kBK) / 64));
-                    uint32_t sfb_bytes = 0;
-#pragma unroll
-                    for (int rb = 0; rb < Cfg::NB; ++rb)
-                        if (int64_t(tc.n_blk) * Cfg::NB + rb < p.n_sf_blocks) sfb_bytes += nsub * 512;
                     mbar_arrive_expect_tx(&full[stage], Cfg::A_BYTES + Cfg::B_BYTES);
-                    mbar_arrive_expect_tx(&sfload[stage], nsub * 512 + sfb_bytes);
-                    tma_load_2d(&tmap_a, &full[stage], smem + Cfg::OFF_A + stage * Cfg::A_BYTES,
+                    // Scales: one box of this k-stage's 8 lines (four 512-byte
+                    // tiles) for the A row block and one for the tile's NB B row
+                    // blocks, counted whole (lines past K, blocks past the
+                    // tensor arrive as zeros).
+                    mbar_arrive_expect_tx(&sfload[stage], Cfg::SFA_BYTES + Cfg::SFB_BYTES);
+                    tma_load_2d(&maps.a, &full[stage], smem + Cfg::OFF_A + stage * Cfg::A_BYTES,
                                 ks * kBKBytes, tc.m_blk * kBM, pol_a);
-                    tma_load_2d(&tmap_b, &full[stage], smem + Cfg::OFF_B + stage * Cfg::B_BYTES,
+                    tma_load_2d(&maps.b, &full[stage], smem + Cfg::OFF_B + stage * Cfg::B_BYTES,
                                 ks * kBKBytes, tc.n_blk * Cfg::BN, pol_b);
-                    bulk_load(smem + Cfg::OFF_SFA + stage * Cfg::SFA_BYTES, asf + ks * 2048,
-                              nsub * 512, &sfload[stage], pol_a);
-#pragma unroll
-                    for (int rb = 0; rb < Cfg::NB; ++rb) {
-                        const int64_t brow = int64_t(tc.n_blk) * Cfg::NB + rb;
-                        if (brow < p.n_sf_blocks)
-                            bulk_load(smem + Cfg::OFF_SFB + stage * Cfg::SFB_BYTES + rb * 2048,
-                                      p.bsf + (brow * kb4 + int64_t(ks) * 4) * 512, nsub * 512,
-                                      &sfload[stage], pol_b);
-                    }
+                    tma_load_3d(&maps.sfa, &sfload[stage], smem + Cfg::OFF_SFA + stage * Cfg::SFA_BYTES,
+                                0, ks * 8, tc.m_blk, pol_a);
+                    tma_load_3d(&maps.sfb, &sfload[stage], smem + Cfg::OFF_SFB + stage * Cfg::SFB_BYTES,
+                                0, ks * 8, tc.n_blk * Cfg::NB, pol_b);
                     if (issued < Cfg::STAGES) ++issued;
                     if (++stage == Cfg::STAGES) {
                         stage = 0;
@@ -436,8 +428,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 }
 
 template <class Cfg, bool kGelu>
-static cudaError_t launch_cfg(const CUtensorMap &ta, const CUtensorMap &tb, const GemmParams &p,
-                              int num_sms, cudaStream_t stream) {
+static cudaError_t launch_cfg(const GemmMaps &maps, const GemmParams &p, int num_sms,
+                              cudaStream_t stream) {
     static int configured_device = -1;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -450,7 +442,7 @@ static cudaError_t launch_cfg(const CUtensorMap &ta, const CUtensorMap &tb, cons
     }
     const int64_t tiles = ((p.M + kBM - 1) / kBM) * ((p.N + Cfg::BN - 1) / Cfg::BN);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-    gemm_kernel<Cfg, kGelu><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
+    gemm_kernel<Cfg, kGelu><<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, stream>>>(maps, p);
     return cudaGetLastError();
 }
 
@@ -483,10 +475,10 @@ cudaError_t launch_gemm(const GemmMaps &maps, const GemmParams &p, GemmKind kind
         return gelu ? launch_pair<true, false>(maps, p, num_sms, stream)
                     : launch_pair<false, false>(maps, p, num_sms, stream);
     if (kind == kGemm256)
-        return gelu ? launch_cfg<Cfg256, true>(maps.a, maps.b, p, num_sms, stream)
-                    : launch_cfg<Cfg256, false>(maps.a, maps.b, p, num_sms, stream);
-    return gelu ? launch_cfg<Cfg128, true>(maps.a, maps.b, p, num_sms, stream)
-                : launch_cfg<Cfg128, false>(maps.a, maps.b, p, num_sms, stream);
+        return gelu ? launch_cfg<Cfg256, true>(maps, p, num_sms, stream)
+                    : launch_cfg<Cfg256, false>(maps, p, num_sms, stream);
+    return gelu ? launch_cfg<Cfg128, true>(maps, p, num_sms, stream)
+                : launch_cfg<Cfg128, false>(maps, p, num_sms, stream);
 }
 
 }  // namespace nvfp4

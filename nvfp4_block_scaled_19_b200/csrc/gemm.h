@@ -9,8 +9,6 @@
 namespace nvfp4 {
 
 struct GemmParams {
-    const uint8_t *asf;     // A scales, tiled layout, pad128(M) x K/16
-    const uint8_t *bsf;     // B scales, tiled layout, pad128(N) x K/16
     const float *a_s_dec;   // 1 fp32
     const float *b_s_dec;   // 1 fp32
     uint8_t *y;             // bf16 [M,N] or null
@@ -23,8 +21,6 @@ struct GemmParams {
     int a_row_scale;        // 1: a_s_dec holds one decode scale per row of A (per token)
     int fp8;                // 1: A and B are E4M3 with per-tensor scales only (no asf/bsf)
     int64_t M, N, K;
-    int64_t n_sf_blocks;    // ceil(N / 128): 128-row blocks present in bsf
-    int64_t m_sf_blocks;    // ceil(M / 128): 128-row blocks present in asf
 };
 
 // Device address of the library's error word (int[2]: code, tag) on the
