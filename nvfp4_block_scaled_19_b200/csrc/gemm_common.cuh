@@ -83,6 +83,8 @@ __device__ __forceinline__ void drain_cols(uint32_t taddr, float alpha, uint32_t
         tmem_ld_32x32b_x32(taddr + ch * 32, r0);
         tmem_ld_32x32b_x32(taddr + ch * 32 + 32, r1);
         tmem_ld_wait();
+        tmem_regs_ready(r0);
+        tmem_regs_ready(r1);
         cvt_32<kGelu>(r0, alpha, pk + 16 * ch);
         cvt_32<kGelu>(r1, alpha, pk + 16 * ch + 16);
     }

@@ -380,6 +380,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                 tmem_ld_32x32b_x32(taddr, r0);
                 tmem_ld_32x32b_x32(taddr + 32, r1);
                 tmem_ld_wait();
+                tmem_regs_ready(r0);
+                tmem_regs_ready(r1);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_l);
