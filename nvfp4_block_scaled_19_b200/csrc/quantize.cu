@@ -20,8 +20,10 @@
 //   word of a small workspace), a bounded grid barrier publishes it, phase 2
 //   quantizes, walking the tensor in the opposite order to phase 1 so that
 //   what phase 1 read last is still in L2 (all of it when the tensor fits).
-//   Rows of a multiple of 64 elements (every DiT shape) take the flat kernel:
-//   the tensor is seen as one array of 16-element blocks, thread g owns
+//   Rows of a multiple of 64 elements (every DiT shape) take the resident
+//   kernel when a slice per SM fits in shared memory (phase 2 then reads the
+//   slice from there, see quantize_dynamic_resident_kernel), else the flat
+//   kernel: the tensor is seen as one array of 16-element blocks, thread g owns
 //   blocks g, g + S, g + 2S, g + 3S of each round (S = threads in the grid),
 //   so every thread has four 32-byte loads in flight in both phases and a
 //   warp's codes are one contiguous 256-byte store.  Other widths take the
@@ -585,6 +587,216 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, const flo
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------
+// quantize_dynamic, resident form: for tensors whose 16-element blocks fit in
+// the shared memory of one CTA per SM (up to ~28 MB of bf16 on 148 SMs; the
+// qkv input of a 1024^2 DiT block is 28.3 MB).  CTA b owns one contiguous
+// slice of whole blocks (a multiple of 4, so a row's four-scale groups never
+// straddle two CTAs) and issues bulk copies of all of it into shared memory
+// at once, in kResPieces pieces with one mbarrier each; the warps of piece p
+// reduce its amax as soon as it lands.  After the grid barrier the slice is
+// quantized from shared memory.  x is read from HBM exactly once, all of it
+// in flight from the start, and phase 2 re-reads nothing from L2.
+
+constexpr int kResThreads = 1024;
+constexpr int kResPieces = 8;
+constexpr int kResWarpsPerPiece = kResThreads / 32 / kResPieces;
+// Shared memory of the slice: leaves room for the static arrays below within
+// the 227 KB a CTA may use.
+constexpr int64_t kResMaxBytes = 216 * 1024;
+
+namespace {
+
+// Bulk-copy and mbarrier helpers of this translation unit (the GEMM's live
+// in ptx.cuh, which only gemm.cu includes).
+__device__ __forceinline__ uint32_t res_smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void res_mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(res_smem_addr(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void res_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(res_smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// Contiguous global -> shared copy (16-byte aligned addresses, size a
+// multiple of 16), completion counted on bar in bytes.
+__device__ __forceinline__ void res_bulk_load(void *dst, const void *src, uint32_t bytes,
+                                              uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            res_smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(res_smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool res_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(res_smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for phase 0 of bar: false once the deadline (%globaltimer
+// ns) has passed.
+__device__ __forceinline__ bool res_wait(uint64_t *bar, uint64_t deadline) {
+    while (!res_try_wait(bar, 0)) {
+        if (globaltimer_ns() > deadline) return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ BF16x16 lds_32B(const uint8_t *p) {
+    BF16x16 v;
+    const uint4 a = *reinterpret_cast<const uint4 *>(p);
+    const uint4 b = *reinterpret_cast<const uint4 *>(p + 16);
+    v.w[0] = a.x; v.w[1] = a.y; v.w[2] = a.z; v.w[3] = a.w;
+    v.w[4] = b.x; v.w[5] = b.y; v.w[6] = b.z; v.w[7] = b.w;
+    return v;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kResThreads, 1) quantize_dynamic_resident_kernel(
+    const uint8_t *__restrict__ x, int64_t rows, int64_t cols, uint32_t per_cta,
+    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, float *__restrict__ s_dec_out,
+    float *__restrict__ amax_out, DynWorkspace *ws, int *err) {
+    extern __shared__ __align__(128) uint8_t xs[];  // the slice, 32 bytes per block
+    __shared__ uint64_t bars[kResPieces];
+    __shared__ unsigned s_amax;
+    __shared__ int s_fail, s_lost;
+    __shared__ uint32_t red[kResThreads / 32];
+    __shared__ float inv_tab[128];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const unsigned long long state0 = tid == 0 ? ld_relaxed_gpu_u64(&ws->state) : 0ull;
+
+    // 32-bit indices: the launch checks that blocks and padded scale
+    // offsets stay below 2^31.
+    const uint32_t kb = static_cast<uint32_t>(cols >> 4);
+    const uint32_t kb4 = kb >> 2;
+    const uint32_t nvec = static_cast<uint32_t>(rows) * kb;  // a multiple of 4
+    const uint32_t lo = min(blockIdx.x * per_cta, nvec);
+    const uint32_t cnt = min(per_cta, nvec - lo);  // a multiple of 4
+    // Piece p: blocks [piece(p), piece(p + 1)) of the slice, multiples of 4.
+    auto piece = [&](int p) -> uint32_t {
+        return p >= kResPieces ? cnt : (cnt / 4 * p / kResPieces) * 4;
+    };
+
+    if (tid == 0) {
+        s_lost = 0;
+        for (int p = 0; p < kResPieces; ++p) res_mbar_init(&bars[p], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (tid == 0) {
+        for (int p = 0; p < kResPieces; ++p) {
+            const uint32_t a = piece(p), bytes = (piece(p + 1) - a) * 32u;
+            res_arrive_expect_tx(&bars[p], bytes);
+            if (bytes != 0) res_bulk_load(xs + 32u * a, x + 32 * (int64_t(lo) + a), bytes, &bars[p]);
+        }
+    }
+
+    // Phase 1: the warps of piece p wait for it, then reduce its amax.
+    uint32_t m = 0;
+    {
+        const int p = warp / kResWarpsPerPiece;
+        const uint32_t t = static_cast<uint32_t>(tid - p * kResWarpsPerPiece * 32);
+        const uint64_t deadline = globaltimer_ns() + kBarrierTimeoutNs;
+        if (res_wait(&bars[p], deadline)) {
+            for (uint32_t i = piece(p) + t; i < piece(p + 1); i += kResWarpsPerPiece * 32)
+                m = max(m, absmax_bf16x16(lds_32B(xs + 32u * i)));
+        } else {
+            s_lost = 1;  // benign race: every writer stores 1
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    if (warp == 0) {
+        m = red[lane];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane == 0) {
+            if (s_lost && err != nullptr && atomicCAS(err, 0, 5) == 0) err[1] = 8;
+            // A CTA whose copies never landed still joins the barrier, so the
+            // others are not left waiting; the error word already says the
+            // result is invalid.
+            unsigned bits = 0;
+            s_fail = grid_amax_barrier(ws, static_cast<unsigned>(state0 >> 32), m, err, &bits) ? 0 : 1;
+            s_amax = bits;
+        }
+    }
+    __syncthreads();
+    if (s_fail || s_lost) {
+        // Copies may still be in flight into this CTA's shared memory: wait
+        // for them (bounded) before the CTA exits.
+        if (tid == 0) {
+            const uint64_t deadline = globaltimer_ns() + kBarrierTimeoutNs;
+            for (int p = 0; p < kResPieces; ++p) res_wait(&bars[p], deadline);
+        }
+        return;
+    }
+    const float amax = __uint_as_float(s_amax);
+    const float s_enc = tensor_encode_scale(amax);
+    if (blockIdx.x == 0 && tid == 0) {
+        if (s_dec_out != nullptr) *s_dec_out = __fdiv_rn(1.0f, s_enc);
+        if (amax_out != nullptr) *amax_out = amax;
+    }
+    fill_inv_table(inv_tab, s_enc);
+    __syncthreads();
+
+    // Phase 2: quantize the slice from shared memory.  Validity is uniform
+    // over each group of 4 lanes (cnt and kResThreads are multiples of 4),
+    // so the scale gather's shuffles see consistent neighbours.
+    for (uint32_t base = 0; base < cnt; base += kResThreads) {
+        const uint32_t i = base + static_cast<uint32_t>(tid);
+        const bool valid = i < cnt;
+        BF16x16 v;
+        if (valid) {
+            v = lds_32B(xs + 32u * i);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v.w[k] = 0u;
+        }
+        const BlockScale bs = block_scale(__uint_as_float(absmax_bf16x16(v) << 16), s_enc, inv_tab);
+        const uint32_t idx = lo + i;
+        if (valid) {
+            const uint4 a = make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]);
+            const uint4 b = make_uint4(v.w[4], v.w[5], v.w[6], v.w[7]);
+            *reinterpret_cast<uint2 *>(q + 8 * static_cast<int64_t>(idx)) =
+                make_uint2(quantize_bf16x8(a, bs.inv), quantize_bf16x8(b, bs.inv));
+        }
+        const uint32_t sfc = valid ? bs.sf : 0u;
+        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sfc, 1);
+        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sfc, 2);
+        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sfc, 3);
+        if (valid && (lane & 3) == 0) {
+            const uint32_t r = idx / kb;
+            const uint32_t c = idx - r * kb;
+            *reinterpret_cast<uint32_t *>(sf + sf_offset(r, c, kb4)) =
+                sfc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        }
+    }
+    // Zero scales of the padding rows [rows, pad128(rows)).
+    const uint32_t rows_i = static_cast<uint32_t>(rows);
+    const uint32_t n_pad = (((rows_i + 127u) & ~127u) - rows_i) * kb4;
+    const uint32_t S = gridDim.x * kResThreads;
+    for (uint32_t i = blockIdx.x * kResThreads + tid; i < n_pad; i += S) {
+        const uint32_t pr = i / kb4;
+        *reinterpret_cast<uint32_t *>(sf + sf_offset(rows_i + pr, 4 * (i - pr * kb4), kb4)) = 0u;
+    }
+}
+
 cudaError_t launch_quantize_dynamic(const void *x, int64_t rows, int64_t cols, uint8_t *q,
                                     uint8_t *sf, float *s_dec_out, float *amax_out,
                                     DynWorkspace *ws, int num_sms, cudaStream_t stream) {
@@ -619,8 +831,36 @@ cudaError_t launch_quantize_dynamic(const void *x, int64_t rows, int64_t cols, u
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (flat) {
-        cfg.gridDim = dim3(grid);
         const uint8_t *xb = reinterpret_cast<const uint8_t *>(x);
+        const int64_t nvec_all = rows * (cols / 16);
+        const int64_t sf_all = ((rows + 127) / 128 * 128) * (cols / 16);
+        // Resident form when one slice per SM fits in shared memory.
+        const int64_t per = ((nvec_all + num_sms - 1) / num_sms + 3) / 4 * 4;
+        if (per * 32 <= kResMaxBytes && nvec_all < (int64_t(1) << 31) &&
+            sf_all < (int64_t(1) << 31)) {
+            static int res_ready[64] = {0};
+            if (!res_ready[dev]) {
+                e = cudaFuncSetAttribute(quantize_dynamic_resident_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kResMaxBytes));
+                if (e != cudaSuccess) return e;
+                int per_sm = 0;
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                    &per_sm, quantize_dynamic_resident_kernel, kResThreads,
+                    static_cast<size_t>(kResMaxBytes));
+                if (e != cudaSuccess) return e;
+                res_ready[dev] = per_sm >= 1 ? 1 : -1;
+            }
+            if (res_ready[dev] == 1) {
+                cfg.gridDim = dim3(num_sms);
+                cfg.blockDim = dim3(kResThreads);
+                cfg.dynamicSmemBytes = static_cast<size_t>(per * 32);
+                return cudaLaunchKernelEx(&cfg, quantize_dynamic_resident_kernel, xb, rows, cols,
+                                          static_cast<uint32_t>(per), q, sf, s_dec_out, amax_out,
+                                          ws, err);
+            }
+        }
+        cfg.gridDim = dim3(grid);
         // 32-bit indices when every index the kernel forms (blocks, padded
         // scale offsets, the last round's overshoot) stays below 2^31.
         const int64_t nvec = rows * (cols / 16);

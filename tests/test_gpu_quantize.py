@@ -158,3 +158,18 @@ def test_quantize_input_16_byte_aligned(nv, path, cols):
     got = (t.q.cpu().numpy(), t.sf.cpu().numpy(), np.float32(t.s_dec.item()),
            np.float32(amax.item()))
     assert_quant_equal(got, oracle_quantize_dynamic(x), f"16B-aligned/{path}")
+
+
+@pytest.mark.parametrize("extra_rows", [0, 1])
+def test_quantize_dynamic_resident_limit(nv, extra_rows):
+    """The single-launch quantize keeps a slice of the input per SM in shared
+    memory when one fits (216 KB of 32-byte blocks, a multiple of 4 blocks);
+    at the largest such input for this GPU and one row past it (the
+    re-reading form) the codes and scales are the oracle's."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cols = 3072
+    kb = cols // 16
+    rows = (sms * (216 * 1024 // 32)) // kb + extra_rows
+    x = draw_x("normal_outliers", rows, cols, seed=rows, index=0)
+    assert_quant_equal(gpu_quantize_dynamic(nv, x, "fused"), oracle_quantize_dynamic(x),
+                       f"{rows}x{cols}")
