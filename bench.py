@@ -459,8 +459,8 @@ def gpu_arm(args) -> dict | None:
                      "note": ("per-token quantize, one pass: algorithmic bytes 2.5625 B/elem "
                               "+ per-row scales" if row else
                               "single-launch amax + dynamic quantize of every layer input; "
-                              "algorithmic bytes 4.5625 B/elem + scales (second read from "
-                              "L2 where the input fits)")},
+                              "algorithmic bytes 4.5625 B/elem + scales (the second read from "
+                              "shared memory where a slice per SM fits, else from L2)")},
         "gemm": {"tflops": round(gemm_tflops, 1), "ms": round(g_avg[top], 5),
                  "layer": layers[top].spec.name},
         "roofline": {"bound": "tensor",
