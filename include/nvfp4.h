@@ -41,6 +41,10 @@
  *    wait records NVFP4_ERR_TIMEOUT in a device word read by
  *    nvfp4_device_error().
  *  - Device pointers must be 16-byte aligned (NVFP4_ERR_MISALIGNED).
+ *  - An empty tensor (rows == 0) is valid input to every quantize call: no
+ *    element is read or written, the arrays of the empty tensor may be NULL,
+ *    and the per-tensor scalars are still written (amax 0, s_dec from the
+ *    scale the call derives or is given).  GEMMs need M, N >= 1.
  *  - The device must be sm_100 (B200); otherwise NVFP4_ERR_UNSUPPORTED_DEVICE.
  *  - Inputs must be finite (no NaN/inf in X or W).
  */
@@ -148,8 +152,9 @@ size_t nvfp4_quantize_dynamic_workspace_bytes(void);
  * the per-16 block quantization of nvfp4_tensor_amax + nvfp4_quantize
  * (nmedialink page above, NVFP4 section: dynamic per-tensor and per-block
  * scales), with identical results.  A cooperative kernel reduces the amax,
- * crosses one grid barrier and quantizes, reading the tensor from L2 the
- * second time where it fits.
+ * crosses one grid barrier and quantizes; where a slice of the tensor per SM
+ * fits in shared memory it stays there between the two phases, otherwise
+ * the second read comes from L2 where the tensor fits.
  *   x_bf16, rows, cols, q_out, sf_out, s_dec_out  as for nvfp4_quantize
  *   amax_out   device, 1 fp32, written with max|x| (NULL = not written)
  *   workspace  device, nvfp4_quantize_dynamic_workspace_bytes() bytes,

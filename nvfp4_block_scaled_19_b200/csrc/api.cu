@@ -121,8 +121,10 @@ nvfp4_status check_quantize_args(const void *x, int64_t rows, int64_t cols, cons
                                  const uint8_t *q, const uint8_t *sf) {
     if (rows < 0 || cols <= 0 || cols % 16 != 0) return NVFP4_ERR_INVALID_ARG;
     if (rows > (int64_t(1) << 40) / cols) return NVFP4_ERR_INVALID_ARG;
-    if (x == nullptr || scale == nullptr || q == nullptr || sf == nullptr)
-        return NVFP4_ERR_INVALID_ARG;
+    if (scale == nullptr) return NVFP4_ERR_INVALID_ARG;
+    // An empty tensor (rows == 0) has no elements to read or write: its
+    // arrays may be NULL.
+    if (rows > 0 && (x == nullptr || q == nullptr || sf == nullptr)) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(q) || !aligned16(sf)) return NVFP4_ERR_MISALIGNED;
     return NVFP4_OK;
 }
@@ -135,7 +137,7 @@ nvfp4_status quantize_impl(const void *x, int64_t rows, int64_t cols, const floa
     int sms = 0;
     st = current_device(&sms);
     if (st != NVFP4_OK) return st;
-    if (rows == 0) return NVFP4_OK;
+    // rows == 0 still launches: the kernel writes s_dec_out from the scale.
     return from_cuda(
         nvfp4::launch_quantize(x, rows, cols, scale, dynamic, q, sf, s_dec_out, sms, stream));
 }
@@ -308,8 +310,8 @@ nvfp4_status nvfp4_fp8_quantize(const void *x_bf16, int64_t rows, int64_t cols,
                                 nvfp4_stream_t stream) {
     if (rows < 0 || cols <= 0 || cols % 16 != 0 || rows > (int64_t(1) << 40) / cols)
         return NVFP4_ERR_INVALID_ARG;
-    if (x_bf16 == nullptr || amax_dev == nullptr || q_out == nullptr || s_dec_out == nullptr)
-        return NVFP4_ERR_INVALID_ARG;
+    if (amax_dev == nullptr || s_dec_out == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (rows > 0 && (x_bf16 == nullptr || q_out == nullptr)) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(x_bf16) || !aligned16(q_out) ||
         (reinterpret_cast<uintptr_t>(amax_dev) & 3u) != 0 ||
         (reinterpret_cast<uintptr_t>(s_dec_out) & 3u) != 0)
@@ -331,6 +333,7 @@ nvfp4_status nvfp4_fp8_gemm(const uint8_t *a8, const float *a_s_dec, const uint8
 nvfp4_status nvfp4_quantize_rowwise(const void *x_bf16, int64_t rows, int64_t cols,
                                     uint8_t *q_out, uint8_t *sf_out, float *s_dec_rows,
                                     float *amax_rows, nvfp4_stream_t stream) {
+    if (rows == 0 && cols > 0 && cols % 16 == 0) return NVFP4_OK;  // no rows, no scales
     nvfp4_status st = check_quantize_args(x_bf16, rows, cols, s_dec_rows, q_out, sf_out);
     if (st != NVFP4_OK) return st;
     if ((reinterpret_cast<uintptr_t>(s_dec_rows) & 3u) != 0 ||

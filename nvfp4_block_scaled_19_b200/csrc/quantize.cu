@@ -571,6 +571,7 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, const flo
     const int64_t target = static_cast<int64_t>(num_sms) * 16;
     const int64_t groups = (rows_pad + kQuantRows - 1) / kQuantRows;
     int64_t gy = (groups + streams_per_cta - 1) / streams_per_cta;
+    if (gy < 1) gy = 1;  // rows == 0: one row of CTAs still writes s_dec_out
     int64_t cap = target / gx;
     if (cap < 1) cap = 1;
     if (gy > cap) gy = cap;

@@ -71,6 +71,10 @@ def test_invalid_arguments_rejected_first(L):
     assert L.nvfp4_quantize(p, 4, 32, p, None, p, None, None) == 1
     assert L.nvfp4_quantize(p + 2, 4, 32, p, p, p, None, None) == 2
     assert L.nvfp4_quantize_with_scale(p, 4, 0, p, p, p, None, None) == 1
+    # an empty tensor's arrays may be NULL (not an argument error); its scale may not
+    assert L.nvfp4_quantize(None, 0, 32, p, None, None, None, None) != 1
+    assert L.nvfp4_quantize(None, 0, 32, None, None, None, None, None) == 1
+    assert L.nvfp4_quantize(None, 4, 32, p, p, p, None, None) == 1
     # amax
     assert L.nvfp4_tensor_amax(p, -5, p, None) == 1
     assert L.nvfp4_tensor_amax(p, 8, None, None) == 1

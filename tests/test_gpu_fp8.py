@@ -96,3 +96,12 @@ def test_gemm_fp8_qkv_full_size_sampled(nv):
     y = _fp8_linear(nv, x, wt)
     ok, worst = oracle.gemm_tolerance_ok(y[rows], _oracle_fp8_linear(x, wt, rows), TOL)
     assert ok, f"qkv fp8: worst {worst:.3f}"
+
+
+def test_quantize_fp8_empty(nv):
+    """0 rows: no codes, S_dec = 1 (amax 0), as the oracle gives."""
+    x = torch.zeros(0, 64, dtype=torch.bfloat16)
+    q, s_dec = _gpu_fp8(nv, x)
+    oq, os_dec, _ = oracle.quantize_fp8(bf16_bits(x), 0, 64)
+    assert q.size == 0 and oq.size == 0
+    assert s_dec == os_dec

@@ -173,3 +173,19 @@ def test_quantize_dynamic_resident_limit(nv, extra_rows):
     x = draw_x("normal_outliers", rows, cols, seed=rows, index=0)
     assert_quant_equal(gpu_quantize_dynamic(nv, x, "fused"), oracle_quantize_dynamic(x),
                        f"{rows}x{cols}")
+
+
+@pytest.mark.parametrize("cols", [64, 80])
+@pytest.mark.parametrize("path", PATHS)
+def test_quantize_empty(nv, orc, cols, path):
+    """An empty tensor (0 rows; its arrays have no storage): no codes, no
+    scales, amax 0 and S_dec = 1 / S_enc(0) = 1 on every path, as the oracle
+    gives; the static-scale call writes 1 / S_enc from its given scale."""
+    x = torch.zeros(0, cols, dtype=torch.bfloat16)
+    assert_quant_equal(gpu_quantize_dynamic(nv, x, path), oracle_quantize_dynamic(x),
+                       f"0x{cols}/{path}")
+    s_enc = torch.tensor([0.37], dtype=torch.float32, device="cuda")
+    t = nv.quantize_with_scale(x.cuda(), s_enc)
+    torch.cuda.synchronize()
+    assert t.q.numel() == 0 and t.sf.numel() == 0
+    assert np.float32(t.s_dec.item()) == orc.decode_scale(np.float32(0.37))

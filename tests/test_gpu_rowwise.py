@@ -96,3 +96,9 @@ def test_gemm_rowscale(nv, M, N, K):
     for m in range(M):
         ok, worst = oracle.gemm_tolerance_ok(yg[m], ref[m], TOL)
         assert ok, f"{M}x{N}x{K} row {m}: worst {worst:.3f}"
+
+
+def test_quantize_rowwise_empty(nv):
+    """0 rows: nothing to quantize and no per-row scales; the call succeeds."""
+    x = torch.zeros(0, 64, dtype=torch.bfloat16)
+    _assert_equal(_gpu_rowwise(nv, x), oracle.quantize_rowwise(bf16_bits(x), 0, 64), "0x64")
