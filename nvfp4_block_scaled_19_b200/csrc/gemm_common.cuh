@@ -33,25 +33,43 @@ __device__ __forceinline__ TileCoord tile_coord(int t, int tiles_m, int tiles_n)
     return c;
 }
 
-// GELU of the fused FFN epilogue, g(h) = 0.5 h (1 + erf(h / sqrt 2)) =
-// 0.5 h erfc(-h / sqrt 2), with erfc(u) for u = |h| / sqrt 2 >= 0 from
-// Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26
-// (Hastings' rational approximation, |error of erf| <= 1.5e-7):
+// GELU of the fused FFN epilogue, g(h) = 0.5 h (1 + erf(h / sqrt 2)), from
+// erfc(u), u = |h| / sqrt 2, by Abramowitz & Stegun, Handbook of
+// Mathematical Functions, formula 7.1.26 (Hastings' rational approximation,
+// |error of erf| <= 1.5e-7):
 //   erfc(u) ~ t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-u^2),
 //   t = 1 / (1 + p u).
-// Then g = 0.5 h c for h < 0 (no cancellation) and g = h - 0.5 h c for
-// h >= 0, with c = erfc(u).  The reciprocal and the exponential use the fast
-// hardware approximations; the total error stays far below the bf16
-// rounding of the output, and about half the instructions of erff.
+// Both signs in one expression without cancellation:
+//   g = max(h, 0) - |h| erfc(|h| / sqrt 2) / 2,
+// (h >= 0: h - h c / 2; h < 0: h c / 2).  Folded at compile time: p / sqrt 2
+// (t straight from |h|), the 1/2 into the coefficients, and exp(-u^2) =
+// 2^(h^2 * (-log2(e) / 2)).  The reciprocal and the power of two are the PTX
+// approximations rcp.approx and ex2.approx (relative errors ~2^-23 and
+// ~2^-22); the total error stays far below the bf16 rounding of the output.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 __device__ __forceinline__ float gelu_erf(float h) {
     constexpr float p = 0.3275911f, a1 = 0.254829592f, a2 = -0.284496736f,
                     a3 = 1.421413741f, a4 = -1.453152027f, a5 = 1.061405429f;
-    const float u = fabsf(h) * 0.70710678118654752f;
-    const float t = __fdividef(1.0f, fmaf(p, u, 1.0f));
-    const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, a5, a4), a3), a2), a1);
-    const float c = poly * __expf(-u * u);
-    const float q = 0.5f * h * c;
-    return h >= 0.0f ? h - q : q;
+    constexpr float p_h = p * 0.70710678118654752f;  // t = 1 / (1 + p_h |h|)
+    constexpr float b1 = 0.5f * a1, b2 = 0.5f * a2, b3 = 0.5f * a3, b4 = 0.5f * a4,
+                    b5 = 0.5f * a5;
+    constexpr float k_e = -0.72134752044448170f;  // -log2(e) / 2
+    const float ah = fabsf(h);
+    const float t = rcp_approx(fmaf(p_h, ah, 1.0f));
+    const float half_c = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, b5, b4), b3), b2), b1) *
+                         ex2_approx(h * h * k_e);
+    return fmaf(-ah, half_c, fmaxf(h, 0.0f));
 }
 
 // Scales 32 fp32 accumulator values by alpha, applies the activation (kGelu)
