@@ -202,10 +202,16 @@ class ClockSampler:
 # ----------------------------------------------------------------- the GPU arm
 
 class Layer:
-    def __init__(self, nv, spec, M, x_cpu, w_cpu, device, row_scales=False, fp8=False):
+    def __init__(self, nv, spec, M, x_cpu, w_cpu, device, row_scales=False, fp8=False,
+                 stale=False):
         self.spec = spec
         self.row_scales = row_scales
         self.fp8 = fp8
+        # One-pass quantize with the previous call's amax: two amax words,
+        # read one and write the other, swapped every call.
+        self.stale = stale and not spec.x_from_prev and not fp8 and not row_scales
+        self.amax_pair = [torch.empty(1, dtype=torch.float32, device=device) for _ in range(2)]
+        self.calls = 0
         if fp8 and spec.x_from_prev:
             raise ValueError("the FP8 variant takes no NVFP4 fused input")
         self.M, self.K = M, spec.K
@@ -222,6 +228,8 @@ class Layer:
             self.xq = (None if spec.x_from_prev
                        else nv.empty_nvfp4(self.M, self.K, device, row_scales=row_scales))
         self.amax = torch.empty(1, dtype=torch.float32, device=device)
+        if self.stale:   # the first call's "previous" amax: this tensor's own
+            nv.tensor_amax(self.x, self.amax_pair[0])
         self.y = (torch.empty(self.M, self.N, dtype=torch.bfloat16, device=device)
                   if spec.keep_y else None)
         self.fused = None
@@ -264,6 +272,8 @@ class Layer:
             return 2 * n + 2 * n + n
         if self.row_scales:   # one pass over X (the second read of a row hits L1/L2)
             return 2 * n + n // 2 + nv.sf_bytes(self.M, self.K) + 4 * self.M
+        if self.stale:        # one pass over X with the previous call's amax
+            return 2 * n + n // 2 + nv.sf_bytes(self.M, self.K)
         return 2 * n + 2 * n + n // 2 + nv.sf_bytes(self.M, self.K)
 
 
@@ -287,6 +297,10 @@ def run_step(nv, layers, ev=None):
             nv.quantize_fp8(L.x, L.amax, L.xq)
         elif L.row_scales:
             nv.quantize_rowwise(L.x, L.xq)
+        elif L.stale:
+            k = L.calls & 1
+            nv.quantize_one_pass(L.x, L.amax_pair[k], L.amax_pair[1 - k], L.xq)
+            L.calls += 1
         else:
             nv.quantize_dynamic(L.x, L.xq, L.amax)
         if ev is not None:
@@ -360,8 +374,9 @@ def gpu_arm(args) -> dict | None:
     peaks, peak_src = load_peaks()
     w = WORKLOADS[args.workload]
     row = args.act_scale == "row"
+    stale = args.act_scale == "stale"
     fp8 = args.variant == "fp8"
-    layers = [Layer(nv, l, w.M, *layer_inputs(w, i), device, row_scales=row, fp8=fp8)
+    layers = [Layer(nv, l, w.M, *layer_inputs(w, i), device, row_scales=row, fp8=fp8, stale=stale)
               for i, l in enumerate(w.layers)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     torch.cuda.synchronize()
@@ -445,6 +460,8 @@ def gpu_arm(args) -> dict | None:
                    "l2": "flushed between steps (256 MiB write, outside the timed spans)",
                    "variant": args.variant,
                    "activation_scale": ("per token (nvfp4_quantize_rowwise, one pass)" if row
+                                        else "per tensor, previous call's amax "
+                                             "(nvfp4_quantize_one_pass, one pass)" if stale
                                         else "per tensor, dynamic (amax + nvfp4_fp8_quantize)"
                                         if fp8 else
                                         "per tensor, dynamic (nvfp4_quantize_dynamic)"),
@@ -458,6 +475,8 @@ def gpu_arm(args) -> dict | None:
                      "ms_per_step": round(q_ms_sum, 5),
                      "note": ("per-token quantize, one pass: algorithmic bytes 2.5625 B/elem "
                               "+ per-row scales" if row else
+                              "one-pass quantize with the previous call's amax: algorithmic "
+                              "bytes 2.5625 B/elem + scales" if stale else
                               "single-launch amax + dynamic quantize of every layer input; "
                               "algorithmic bytes 4.5625 B/elem + scales (the second read from "
                               "shared memory where a slice per SM fits, else from L2)")},
@@ -488,7 +507,7 @@ def host_e2e(nv, layers, args, device, dist, world) -> dict:
     Independent layers go through nvfp4_linear_host; a chain (a layer fed by
     the previous layer's fused output) through the Python API, copying every
     drawn X in and the last layer's Y out."""
-    if any(L.spec.x_from_prev or L.row_scales or L.fp8 for L in layers):
+    if any(L.spec.x_from_prev or L.row_scales or L.fp8 or L.stale for L in layers):
         return chain_e2e(nv, layers, args, device, dist, world)
     stream = torch.cuda.current_stream()
     hosts = []
@@ -547,7 +566,8 @@ def chain_e2e(nv, layers, args, device, dist, world) -> dict:
     return {"value": round(aggregate(flops, world, sec) / 1e12, 3), "unit": UNIT,
             "h2d_bytes_per_step": sum(L.M * L.K * 2 for L, _ in xs),
             "d2h_bytes_per_step": sum(L.M * L.N * 2 for L, _ in ys), "steps": steps,
-            "api": "Python API (quantize_dynamic / quantize_rowwise / quantize_fp8, gemm), "
+            "api": "Python API (quantize_dynamic / quantize_rowwise / quantize_one_pass / "
+                   "quantize_fp8, gemm), "
                    "pinned host buffers"}
 
 
@@ -649,8 +669,9 @@ def main(argv=None) -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", choices=["nvfp4", "fp8"], default="nvfp4",
                     help="nvfp4 (the path) or the FP8 per-tensor variant")
-    ap.add_argument("--act-scale", choices=["tensor", "row"], default="tensor",
-                    help="activation tensor scale: per tensor (the pages' scheme) or per token")
+    ap.add_argument("--act-scale", choices=["tensor", "row", "stale"], default="tensor",
+                    help="activation tensor scale: per tensor (the pages' scheme), per token, "
+                         "or per tensor from the previous call's amax (one pass)")
     args = ap.parse_args(argv)
     line = reference_arm(args) if args.impl == "reference" else gpu_arm(args)
     if line is not None:

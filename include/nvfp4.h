@@ -145,6 +145,22 @@ nvfp4_status nvfp4_quantize_with_scale(const void *x_bf16, int64_t rows, int64_t
                                        uint8_t *sf_out, float *s_dec_out,
                                        nvfp4_stream_t stream);
 
+/* One-pass NVFP4 quantization with the tensor scale of an earlier tensor:
+ * the per-tensor scale "static or dynamic" (nmedialink page above, NVFP4
+ * section) read as dynamic but one call stale.  S_enc is derived on the
+ * device from *amax_prev_dev exactly as nvfp4_quantize derives it from
+ * *amax_dev, the tensor is read once (no amax pass before the quantize),
+ * and this tensor's own amax is written for the next call.  Blocks whose
+ * values outgrew the stale scale saturate (E4M3 448, E2M1 6).
+ *   x_bf16, rows, cols, q_out, sf_out, s_dec_out  as for nvfp4_quantize
+ *   amax_prev_dev  device, 1 fp32, read (an earlier call's amax_out, or any
+ *                  amax the caller chooses for the first call)
+ *   amax_out       device, 1 fp32, written with max|x| of this tensor; must
+ *                  not alias amax_prev_dev (callers alternate two words) */
+nvfp4_status nvfp4_quantize_one_pass(const void *x_bf16, int64_t rows, int64_t cols,
+                                     const float *amax_prev_dev, uint8_t *q_out, uint8_t *sf_out,
+                                     float *s_dec_out, float *amax_out, nvfp4_stream_t stream);
+
 /* Bytes of device workspace needed by nvfp4_quantize_dynamic (32). */
 size_t nvfp4_quantize_dynamic_workspace_bytes(void);
 

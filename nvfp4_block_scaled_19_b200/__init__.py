@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_quantize.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
         L.nvfp4_quantize_with_scale.restype = st
         L.nvfp4_quantize_with_scale.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
+        L.nvfp4_quantize_one_pass.restype = st
+        L.nvfp4_quantize_one_pass.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp, vp]
         L.nvfp4_quantize_dynamic_workspace_bytes.restype = ctypes.c_size_t
         L.nvfp4_quantize_dynamic_workspace_bytes.argtypes = []
         L.nvfp4_quantize_dynamic.restype = st
@@ -175,6 +177,20 @@ def quantize_with_scale(x: torch.Tensor, s_enc: torch.Tensor, out: NVFP4Tensor |
     _check("nvfp4_quantize_with_scale", lib().nvfp4_quantize_with_scale(
         x.data_ptr(), rows, cols, s_enc.data_ptr(), out.q.data_ptr(), out.sf.data_ptr(),
         out.s_dec.data_ptr(), _stream(stream)))
+    return out
+
+
+def quantize_one_pass(x: torch.Tensor, amax_prev: torch.Tensor, amax_out: torch.Tensor,
+                      out: NVFP4Tensor | None = None, stream=None) -> NVFP4Tensor:
+    """One pass over x with the tensor scale derived from an earlier amax
+    (amax_prev, device fp32); writes this tensor's amax into amax_out (a
+    different device fp32) for the next call."""
+    _require(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    out = empty_nvfp4(rows, cols, x.device) if out is None else out
+    _check("nvfp4_quantize_one_pass", lib().nvfp4_quantize_one_pass(
+        x.data_ptr(), rows, cols, amax_prev.data_ptr(), out.q.data_ptr(), out.sf.data_ptr(),
+        out.s_dec.data_ptr(), amax_out.data_ptr(), _stream(stream)))
     return out
 
 

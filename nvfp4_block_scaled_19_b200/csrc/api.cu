@@ -193,6 +193,20 @@ nvfp4_status nvfp4_quantize_with_scale(const void *x_bf16, int64_t rows, int64_t
     return quantize_impl(x_bf16, rows, cols, s_enc_dev, false, q_out, sf_out, s_dec_out, stream);
 }
 
+nvfp4_status nvfp4_quantize_one_pass(const void *x_bf16, int64_t rows, int64_t cols,
+                                     const float *amax_prev_dev, uint8_t *q_out, uint8_t *sf_out,
+                                     float *s_dec_out, float *amax_out, nvfp4_stream_t stream) {
+    nvfp4_status st = check_quantize_args(x_bf16, rows, cols, amax_prev_dev, q_out, sf_out);
+    if (st != NVFP4_OK) return st;
+    if (amax_out == nullptr || amax_out == amax_prev_dev) return NVFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(amax_out) & 3u) != 0) return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(nvfp4::launch_quantize(x_bf16, rows, cols, amax_prev_dev, true, q_out, sf_out,
+                                            s_dec_out, sms, stream, amax_out));
+}
+
 size_t nvfp4_quantize_dynamic_workspace_bytes(void) { return sizeof(nvfp4::DynWorkspace); }
 
 nvfp4_status nvfp4_quantize_dynamic(const void *x_bf16, int64_t rows, int64_t cols, uint8_t *q_out,

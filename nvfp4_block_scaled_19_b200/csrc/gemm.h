@@ -49,9 +49,10 @@ cudaError_t launch_gemm(const GemmMaps &maps, const GemmParams &p, GemmKind kind
 cudaError_t launch_amax(const void *x, int64_t numel, float *amax, int num_sms,
                         cudaStream_t stream);
 
+// amax_out (optional): also writes max |x| of this tensor (one pass).
 cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, const float *scale_in,
                             bool dynamic, uint8_t *q, uint8_t *sf, float *s_dec_out, int num_sms,
-                            cudaStream_t stream);
+                            cudaStream_t stream, float *amax_out = nullptr);
 
 // Workspace of the single-launch dynamic quantization (zero-initialised once
 // by the caller; calls that share one must be stream-ordered).

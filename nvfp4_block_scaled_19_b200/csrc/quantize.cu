@@ -86,7 +86,7 @@ constexpr int kQuantRows = 2;       // rows per group; the next group is loaded 
 // flight while the current one is computed.  Covers the padded scale layout:
 // rows up to a multiple of 128 and block columns up to a multiple of 4 get
 // zero scales.  All 32 lanes of a warp share (bx, rs), so shuffles are uniform.
-__device__ __forceinline__ void quantize_rows(const uint16_t *__restrict__ x, int64_t rows,
+__device__ __forceinline__ uint32_t quantize_rows(const uint16_t *__restrict__ x, int64_t rows,
                                               int64_t cols, float s_enc, const float *inv_tab,
                                               uint8_t *__restrict__ q, uint8_t *__restrict__ sf,
                                               int bx, int64_t rs, int64_t n_streams, int tx,
@@ -117,8 +117,9 @@ __device__ __forceinline__ void quantize_rows(const uint16_t *__restrict__ x, in
         }
     };
 
+    uint32_t amax_bits = 0;  // running |x| maximum of this thread's blocks (bf16 bits)
     int64_t g = rs;
-    if (g >= n_groups) return;
+    if (g >= n_groups) return amax_bits;
     BF16x16 cur[kQuantRows];
     load(row_of(g), cur);
     while (true) {
@@ -131,8 +132,9 @@ __device__ __forceinline__ void quantize_rows(const uint16_t *__restrict__ x, in
             const int64_t r = r0 + u;
             if (r >= rows_pad) break;  // uniform across the warp
             const bool valid = r < rows && col_ok;
-            const BlockScale bs =
-                block_scale(__uint_as_float(absmax_bf16x16(cur[u]) << 16), s_enc, inv_tab);
+            const uint32_t mb = absmax_bf16x16(cur[u]);  // 0 for padding (zero-filled)
+            amax_bits = max(amax_bits, mb);
+            const BlockScale bs = block_scale(__uint_as_float(mb << 16), s_enc, inv_tab);
             const uint32_t sfc = valid ? bs.sf : 0u;
             if (valid) {
                 const uint4 lo = make_uint4(cur[u].w[0], cur[u].w[1], cur[u].w[2], cur[u].w[3]);
@@ -152,14 +154,19 @@ __device__ __forceinline__ void quantize_rows(const uint16_t *__restrict__ x, in
 #pragma unroll
         for (int u = 0; u < kQuantRows; ++u) cur[u] = nxt[u];
     }
+    return amax_bits;
 }
 
 // grid.x covers the padded block columns (64 per slice), grid.y x 2 row
 // streams stride the rows.
+// amax_out (optional, zeroed by the launch): max |x| of this tensor, folded
+// in with one atomicMax per warp on the float's bit pattern; the one-pass
+// quantize with an earlier call's scale hands it to the next call.
 template <bool kDynamic>
 __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(
     const uint16_t *__restrict__ x, int64_t rows, int64_t cols, const float *__restrict__ scale_in,
-    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, float *__restrict__ s_dec_out) {
+    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, float *__restrict__ s_dec_out,
+    unsigned *__restrict__ amax_out) {
     const float s_enc = kDynamic ? tensor_encode_scale(*scale_in) : *scale_in;
     if (s_dec_out != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
         *s_dec_out = __fdiv_rn(1.0f, s_enc);
@@ -167,9 +174,15 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(
     fill_inv_table(inv_tab, s_enc);
     __syncthreads();
     constexpr int kStreams = kQuantThreads / kSliceBlocks;
-    quantize_rows(x, rows, cols, s_enc, inv_tab, q, sf, blockIdx.x,
-                  static_cast<int64_t>(blockIdx.y) * kStreams + threadIdx.x / kSliceBlocks,
-                  static_cast<int64_t>(gridDim.y) * kStreams, threadIdx.x % kSliceBlocks, false);
+    uint32_t m = quantize_rows(x, rows, cols, s_enc, inv_tab, q, sf, blockIdx.x,
+                               static_cast<int64_t>(blockIdx.y) * kStreams + threadIdx.x / kSliceBlocks,
+                               static_cast<int64_t>(gridDim.y) * kStreams, threadIdx.x % kSliceBlocks,
+                               false);
+    if (amax_out != nullptr) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(amax_out, m << 16);
+    }
 }
 
 constexpr int kDynThreads = 512;  // 4 row streams x 128 threads
@@ -563,7 +576,11 @@ cudaError_t launch_amax(const void *x, int64_t numel, float *amax, int num_sms,
 
 cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, const float *scale_in,
                             bool dynamic, uint8_t *q, uint8_t *sf, float *s_dec_out, int num_sms,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, float *amax_out) {
+    if (amax_out != nullptr) {
+        const cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), stream);
+        if (e != cudaSuccess) return e;
+    }
     const int64_t kbp = ((cols / 16 + 3) / 4) * 4;
     const int64_t rows_pad = (rows + 127) / 128 * 128;
     const int64_t gx = (kbp + kSliceBlocks - 1) / kSliceBlocks;
@@ -579,12 +596,13 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, const flo
     if (gx > 2147483647) return cudaErrorInvalidValue;
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
     const uint16_t *xp = reinterpret_cast<const uint16_t *>(x);
+    unsigned *am = reinterpret_cast<unsigned *>(amax_out);
     if (dynamic)
         quantize_kernel<true><<<grid, kQuantThreads, 0, stream>>>(xp, rows, cols, scale_in, q, sf,
-                                                                 s_dec_out);
+                                                                 s_dec_out, am);
     else
         quantize_kernel<false><<<grid, kQuantThreads, 0, stream>>>(xp, rows, cols, scale_in, q,
-                                                                  sf, s_dec_out);
+                                                                  sf, s_dec_out, am);
     return cudaGetLastError();
 }
 

@@ -145,6 +145,17 @@ def quantize_dynamic(x_bits: np.ndarray, rows: int, cols: int):
     return q, sf, decode_scale(s_enc), amax
 
 
+def quantize_one_pass(x_bits: np.ndarray, rows: int, cols: int, amax_prev):
+    """The per-tensor scale one call stale: S_enc from an earlier tensor's
+    amax (the "static or dynamic" FP32 scale of the NVFP4 section of the
+    nmedialink page, read as dynamic with the previous call's amax), then the
+    same block quantize; returns (q, sf, s_dec, amax of this tensor for the
+    next call)."""
+    s_enc = tensor_scale(amax_prev)
+    q, sf = quantize(x_bits, rows, cols, s_enc)
+    return q, sf, decode_scale(s_enc), tensor_amax(x_bits)
+
+
 def dequantize(q: np.ndarray, sf: np.ndarray, s_dec, rows: int, cols: int,
                row_idx: np.ndarray | None = None) -> np.ndarray:
     """fp64 x_hat = e2m1(q) * e4m3(sf) * s_dec for all rows or the listed ones."""

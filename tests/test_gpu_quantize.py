@@ -189,3 +189,31 @@ def test_quantize_empty(nv, orc, cols, path):
     torch.cuda.synchronize()
     assert t.q.numel() == 0 and t.sf.numel() == 0
     assert np.float32(t.s_dec.item()) == orc.decode_scale(np.float32(0.37))
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 16), (130, 272), (257, 512), (64, 3072), (4608, 3072)])
+@pytest.mark.parametrize("prev", [0.5, 1.0, 1.3])
+def test_quantize_one_pass(nv, orc, rows, cols, prev):
+    """One pass with the scale from an earlier amax (prev x this tensor's:
+    saturating, exact, with headroom): codes, scales and S_dec are the
+    oracle's for that amax, and the amax written for the next call is this
+    tensor's."""
+    x = draw_x("normal_outliers", rows, cols, seed=rows + cols, index=0)
+    xb = bf16_bits(x)
+    amax_prev = np.float32(orc.tensor_amax(xb) * np.float32(prev))
+    a_prev = torch.tensor([float(amax_prev)], dtype=torch.float32, device="cuda")
+    a_out = torch.full((1,), -1.0, device="cuda")
+    t = nv.quantize_one_pass(x.cuda(), a_prev, a_out)
+    torch.cuda.synchronize()
+    oq, osf, osd, oamax = orc.quantize_one_pass(xb, rows, cols, amax_prev)
+    assert np.array_equal(t.q.cpu().numpy(), oq)
+    assert np.array_equal(t.sf.cpu().numpy(), osf)
+    assert np.float32(t.s_dec.item()) == osd
+    assert np.float32(a_out.item()) == oamax
+
+
+def test_quantize_one_pass_rejects_aliased_amax(nv):
+    x = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    a = torch.ones(1, device="cuda")
+    with pytest.raises(nv.NVFP4Error):
+        nv.quantize_one_pass(x, a, a)
