@@ -625,6 +625,59 @@ def cpu_baseline(w, target_s: float) -> dict:
             "sample": f"{passes} passes of: {desc}", "seconds": round(secs, 3)}
 
 
+def quantize_sweep(args) -> dict:
+    """Quantize throughput over sizes: 2^20 .. 2^29 bf16 elements as
+    [n / 4096, 4096] N(0,1) (seeded, drawn on the device), each path timed
+    with CUDA events over `sweep_iters` calls, L2 flushed (256 MiB write)
+    before every call, outside the timed span.  Algorithmic bytes: dynamic
+    4.5625 B/elem (amax read + quantize read + codes and scales written),
+    one pass 2.5625 B/elem, amax alone 2 B/elem."""
+    import nvfp4_block_scaled_19_b200 as nv
+    torch.cuda.set_device(0)
+    peaks, _ = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    gen = torch.Generator(device="cuda")
+    rows_out = []
+    for lg in range(20, 30):
+        n = 1 << lg
+        gen.manual_seed(lg)
+        x = torch.randn(n // 4096, 4096, generator=gen, device="cuda").to(torch.bfloat16)
+        out = nv.empty_nvfp4(n // 4096, 4096)
+        amax = torch.empty(1, device="cuda")
+        a_pair = [torch.empty(1, device="cuda") for _ in range(2)]
+        nv.tensor_amax(x, a_pair[0])
+        paths = {
+            "dynamic": (lambda: nv.quantize_dynamic(x, out, amax), 4.5625),
+            "one_pass_stale": (lambda: nv.quantize_one_pass(x, a_pair[0], a_pair[1], out), 2.5625),
+            "amax": (lambda: nv.tensor_amax(x, amax), 2.0),
+        }
+        row = {"elements": n, "shape": [n // 4096, 4096]}
+        for name, (fn, bpe) in paths.items():
+            for _ in range(3):
+                fn()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.sweep_iters)]
+            for e0, e1 in ev:
+                flush.zero_()
+                e0.record()
+                fn()
+                e1.record()
+            torch.cuda.synchronize()
+            us = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev) * 1e3
+            gbs = n * bpe / (us * 1e-6) / 1e9
+            row[name] = {"us": round(us, 2), "gbs": round(gbs, 1), "pct_hbm": round(gbs / hbm, 4)}
+        rows_out.append(row)
+        del x, out
+    code, detail = nv.device_error()
+    if code != 0:
+        raise RuntimeError(f"device wait timed out (tag {detail})")
+    return {"metric": "quantize GB/s (% HBM) over sizes", "unit": "GB/s", "hbm_gbs": hbm,
+            "data": "synthetic N(0,1), seeded on the device", "iters": args.sweep_iters,
+            "l2": "flushed before every call (256 MiB write, outside the timed span)",
+            "sweep": rows_out}
+
+
 def reference_arm(args) -> dict | None:
     rank, world, _ = dist_env()
     if rank != 0:
@@ -672,7 +725,13 @@ def main(argv=None) -> int:
     ap.add_argument("--act-scale", choices=["tensor", "row", "stale"], default="tensor",
                     help="activation tensor scale: per tensor (the pages' scheme), per token, "
                          "or per tensor from the previous call's amax (one pass)")
+    ap.add_argument("--quantize-sweep", action="store_true",
+                    help="instead of the step: quantize throughput over 2^20..2^29 elements")
+    ap.add_argument("--sweep-iters", type=int, default=20)
     args = ap.parse_args(argv)
+    if args.quantize_sweep:
+        print(json.dumps(quantize_sweep(args)), flush=True)
+        return 0
     line = reference_arm(args) if args.impl == "reference" else gpu_arm(args)
     if line is not None:
         print(json.dumps(line), flush=True)

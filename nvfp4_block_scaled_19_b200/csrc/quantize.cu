@@ -574,12 +574,125 @@ cudaError_t launch_amax(const void *x, int64_t numel, float *amax, int num_sms,
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------
+// One-pass block quantize with S_enc known before the pass (given, or derived
+// from an amax the caller holds), for rows of a multiple of 64 elements: the
+// flat layout of quantize_dynamic_flat_kernel's phase 2 without its amax
+// phase and grid barrier.  Thread g of S quantizes blocks g, g+S, g+2S, g+3S
+// of every round of 4S blocks, all four loads in flight; optionally folds
+// max |x| into amax_out (zeroed by the launch) for a later call.
+template <bool kDynamic, typename Idx>
+__global__ void __launch_bounds__(kFlatThreads, 2) quantize_flat_kernel(
+    const uint8_t *__restrict__ x, int64_t rows, int64_t cols, const float *__restrict__ scale_in,
+    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, float *__restrict__ s_dec_out,
+    unsigned *__restrict__ amax_out) {
+    __shared__ float inv_tab[128];
+    const int tid = threadIdx.x, lane = tid & 31;
+    const float s_enc = kDynamic ? tensor_encode_scale(*scale_in) : *scale_in;
+    if (s_dec_out != nullptr && blockIdx.x == 0 && tid == 0) *s_dec_out = __fdiv_rn(1.0f, s_enc);
+    fill_inv_table(inv_tab, s_enc);
+    __syncthreads();
+
+    const bool a32 = (reinterpret_cast<uintptr_t>(x) & 31) == 0;
+    const Idx kb = static_cast<Idx>(cols >> 4);
+    const Idx kb4 = kb >> 2;
+    const Idx nvec = static_cast<Idx>(rows) * kb;  // a multiple of 4
+    const Idx S = static_cast<Idx>(gridDim.x) * kFlatThreads;
+    const Idx chunk = S * kFlatU;
+    const Idx g = static_cast<Idx>(blockIdx.x) * kFlatThreads + tid;
+    const Idx n_rounds = (nvec + chunk - 1) / chunk;
+    uint32_t m = 0;
+    for (Idx rd = 0; rd < n_rounds; ++rd) {
+        BF16x16 v[kFlatU];
+#pragma unroll
+        for (int u = 0; u < kFlatU; ++u) {
+            const Idx idx = rd * chunk + u * S + g;
+            if (idx < nvec) {
+                v[u] = ldg_32B(x + 32 * static_cast<int64_t>(idx), a32);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[u].w[k] = 0u;
+            }
+        }
+        // Validity is uniform over each group of 4 lanes (nvec, S and every
+        // warp's first index are multiples of 4).
+#pragma unroll
+        for (int u = 0; u < kFlatU; ++u) {
+            const Idx idx = rd * chunk + u * S + g;
+            const bool valid = idx < nvec;
+            const uint32_t mb = absmax_bf16x16(v[u]);
+            m = max(m, mb);
+            const BlockScale bs = block_scale(__uint_as_float(mb << 16), s_enc, inv_tab);
+            if (valid) {
+                const uint4 lo = make_uint4(v[u].w[0], v[u].w[1], v[u].w[2], v[u].w[3]);
+                const uint4 hi = make_uint4(v[u].w[4], v[u].w[5], v[u].w[6], v[u].w[7]);
+                *reinterpret_cast<uint2 *>(q + 8 * static_cast<int64_t>(idx)) =
+                    make_uint2(quantize_bf16x8(lo, bs.inv), quantize_bf16x8(hi, bs.inv));
+            }
+            const uint32_t sfc = valid ? bs.sf : 0u;
+            const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sfc, 1);
+            const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sfc, 2);
+            const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sfc, 3);
+            if (valid && (lane & 3) == 0) {
+                const Idx r = idx / kb;
+                const Idx c = idx - r * kb;
+                *reinterpret_cast<uint32_t *>(sf + sf_offset(r, c, kb4)) =
+                    sfc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            }
+        }
+    }
+    // Zero scales of the padding rows [rows, pad128(rows)).
+    const Idx rows_i = static_cast<Idx>(rows);
+    const Idx n_pad = (((rows_i + 127) & ~Idx(127)) - rows_i) * kb4;
+    for (Idx i = g; i < n_pad; i += S) {
+        const Idx pr = i / kb4;
+        *reinterpret_cast<uint32_t *>(sf + sf_offset(rows_i + pr, 4 * (i - pr * kb4), kb4)) = 0u;
+    }
+    if (amax_out != nullptr) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+        if (lane == 0 && m != 0) atomicMax(amax_out, m << 16);
+    }
+}
+
 cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, const float *scale_in,
                             bool dynamic, uint8_t *q, uint8_t *sf, float *s_dec_out, int num_sms,
                             cudaStream_t stream, float *amax_out) {
     if (amax_out != nullptr) {
         const cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), stream);
         if (e != cudaSuccess) return e;
+    }
+    unsigned *am = reinterpret_cast<unsigned *>(amax_out);
+    if (cols % 64 == 0) {
+        // Flat one-pass kernel: up to 2 CTAs per SM, at least ~one block per
+        // thread; 32-bit indices where every index (blocks, padded scale
+        // offsets, the last round's overshoot) stays below 2^31.
+        const int64_t nvec = rows * (cols / 16);
+        int64_t grid = (nvec + kFlatThreads - 1) / kFlatThreads;
+        const int64_t cap = static_cast<int64_t>(num_sms) * 2;
+        if (grid > cap) grid = cap;
+        if (grid < 1) grid = 1;
+        const int64_t span = grid * kFlatThreads * kFlatU;
+        const int64_t sf_span = ((rows + 127) / 128 * 128) * (cols / 16);
+        const uint8_t *xb = reinterpret_cast<const uint8_t *>(x);
+        const unsigned gs = static_cast<unsigned>(grid);
+        const bool narrow = nvec + span < (int64_t(1) << 31) && sf_span < (int64_t(1) << 31);
+        if (dynamic) {
+            if (narrow)
+                quantize_flat_kernel<true, uint32_t><<<gs, kFlatThreads, 0, stream>>>(
+                    xb, rows, cols, scale_in, q, sf, s_dec_out, am);
+            else
+                quantize_flat_kernel<true, int64_t><<<gs, kFlatThreads, 0, stream>>>(
+                    xb, rows, cols, scale_in, q, sf, s_dec_out, am);
+        } else {
+            if (narrow)
+                quantize_flat_kernel<false, uint32_t><<<gs, kFlatThreads, 0, stream>>>(
+                    xb, rows, cols, scale_in, q, sf, s_dec_out, am);
+            else
+                quantize_flat_kernel<false, int64_t><<<gs, kFlatThreads, 0, stream>>>(
+                    xb, rows, cols, scale_in, q, sf, s_dec_out, am);
+        }
+        return cudaGetLastError();
     }
     const int64_t kbp = ((cols / 16 + 3) / 4) * 4;
     const int64_t rows_pad = (rows + 127) / 128 * 128;
@@ -596,7 +709,6 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, const flo
     if (gx > 2147483647) return cudaErrorInvalidValue;
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
     const uint16_t *xp = reinterpret_cast<const uint16_t *>(x);
-    unsigned *am = reinterpret_cast<unsigned *>(amax_out);
     if (dynamic)
         quantize_kernel<true><<<grid, kQuantThreads, 0, stream>>>(xp, rows, cols, scale_in, q, sf,
                                                                  s_dec_out, am);
