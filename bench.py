@@ -51,14 +51,39 @@ GEMM_SOURCES = ["gemm.h", "gemm.cu", "gemm_pair.cuh", "gemm_common.cuh", "ptx.cu
                 "nvfp4_math.cuh"]
 
 
+def strip_c_comments(text: str) -> str:
+    """C/C++ source without its comments, whitespace runs collapsed to one
+    space (string and character literals kept as written)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def gemm_source_hash() -> str:
-    """sha256 over the GEMM kernel sources, in a fixed order: ties a profile's
-    counters to the kernel they were taken on."""
+    """sha256 over the GEMM kernel sources without their comments, in a fixed
+    order: ties a profile's counters to the kernel code they were taken on."""
     import hashlib
     h = hashlib.sha256()
     for name in GEMM_SOURCES:
-        with open(os.path.join(ROOT, "nvfp4_block_scaled_19_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "nvfp4_block_scaled_19_b200", "csrc", name)) as f:
+            h.update(strip_c_comments(f.read()).encode())
     return h.hexdigest()
 
 

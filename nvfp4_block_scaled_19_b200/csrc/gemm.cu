@@ -10,9 +10,10 @@
 // Design (persistent, warp-specialised, one CTA per SM, 128 x BN tiles):
 //   warp 0        TMA producer: per k-stage of 256 elements, a 2-D TMA load of
 //                 the A tile (128 rows x 128 B, 128B swizzle), one of the B
-//                 tile (BN rows), and contiguous bulk copies of the matching
-//                 scale factors (the 128x4-tiled layout makes a 128-row x
-//                 256-K slice one contiguous 2 KB run).  No multicast.
+//                 tile (BN rows), and one 3-D TMA box per operand of the
+//                 matching scale factors (the 128x4-tiled layout makes a
+//                 128-row x 256-K slice one contiguous 2 KB run: 8 lines of
+//                 256 bytes per 128-row block).  No multicast.
 //   warp 1        MMA issuer (one thread): four tcgen05.mma kind::mxf4nvf4
 //                 block_scale scale_vec::4X (K = 64 each) per stage into the
 //                 tile's TMEM accumulator; tcgen05.commit frees the stage and,

@@ -14,8 +14,9 @@
 //              `full` barrier with both CTAs' A+B bytes; each CTA issues
 //              `.cta_group::2` TMA loads (no multicast) of its A and B halves
 //              into its own shared memory that complete on the leader's
-//              `full` barrier, and bulk-copies its scale factors (its 128 A
-//              rows, all 256 B rows) against its own `sfload` barrier.
+//              `full` barrier, and loads its scale factors (its 128 A rows,
+//              all 256 B rows: one 3-D TMA box each) against its own
+//              `sfload` barrier.
 //   warp 1     leader only: issues the MMAs (cta_group::2) and commits to the
 //              `empty`, `acc_full` barriers of both CTAs (tcgen05.commit
 //              multicast); both CTAs' warp 1 allocate / free the TMEM pair.
