@@ -1,0 +1,53 @@
+"""bench.py's JSON line keeps the contract: the keys and their meaning on
+both arms (the oracle's reference arm runs here, the GPU arm on a B200)."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+BASE_KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+             "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config"}
+
+
+def _run(args, timeout):
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT,
+                       capture_output=True, text=True, timeout=timeout)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+def test_reference_arm_line():
+    d = _run(["--impl", "reference", "--steps", "2", "--warmup", "1", "--cpu-seconds", "0.5"], 300)
+    assert BASE_KEYS <= set(d)
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["n_gpus"] == 1
+    assert d["config"]["workload"] == "qkv_1024" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+@pytest.mark.gpu
+def test_gpu_arm_line():
+    d = _run(["--steps", "20", "--warmup", "3", "--no-cpu-baseline", "--e2e-steps", "2"], 600)
+    assert BASE_KEYS <= set(d)
+    assert d["n_gpus"] == 1 and d["steps"] == 20 and d["warmup"] == 3
+    assert d["higher_is_better"] is True and d["scaling"] == "weak"
+    assert d["config"]["workload"] == "qkv_1024"
+    r = d["roofline"]
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert 0 < r["frac"] < 1.5 and abs(r["achieved"] / r["peak"] - r["frac"]) < 1e-3
+    assert r["traffic"] is None or r["traffic"] > 0
+    e = d["e2e"]
+    assert e["h2d_bytes_per_step"] == 4608 * 3072 * 2 and e["d2h_bytes_per_step"] == 4608 * 9216 * 2
+    assert 0 < e["value"] < d["value"]
+    assert d["gpu_launches"] == 2 * 20
+    assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(d["clocks"])
+    # ms_per_step is the evented step; value is the work of the step over it
+    assert abs(2 * 4608 * 9216 * 3072 / (d["ms_per_step"] * 1e-3) / 1e12 - d["value"]) \
+        < 0.01 * d["value"]
