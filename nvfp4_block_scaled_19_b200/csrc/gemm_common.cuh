@@ -58,34 +58,47 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return r;
 }
 
-__device__ __forceinline__ float gelu_erf(float h) {
-    constexpr float p = 0.3275911f, a1 = 0.254829592f, a2 = -0.284496736f,
-                    a3 = 1.421413741f, a4 = -1.453152027f, a5 = 1.061405429f;
-    constexpr float p_h = p * 0.70710678118654752f;  // t = 1 / (1 + p_h |h|)
-    constexpr float b1 = 0.5f * a1, b2 = 0.5f * a2, b3 = 0.5f * a3, b4 = 0.5f * a4,
-                    b5 = 0.5f * a5;
+// Abramowitz & Stegun 7.1.26, published coefficients.
+constexpr float kAsP = 0.3275911f, kAsA1 = 0.254829592f, kAsA2 = -0.284496736f,
+                kAsA3 = 1.421413741f, kAsA4 = -1.453152027f, kAsA5 = 1.061405429f;
+
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+
+// GELU of two values with the packed f32x2 operations of sm_100 (two fp32
+// FMAs or products, each rounded as its scalar form, per instruction): the
+// result is bit-identical to the scalar arrangement g = fma(-|h|, c/2,
+// max(h, 0)) with c/2 = (t * poly) * e, because the -1/2 is folded into the
+// coefficients (negating every coefficient negates every rounded
+// intermediate exactly).
+__device__ __forceinline__ float2 gelu_erf2(float2 h) {
+    constexpr float p_h = kAsP * 0.70710678118654752f;  // t = 1 / (1 + p_h |h|)
+    constexpr float n1 = -0.5f * kAsA1, n2 = -0.5f * kAsA2, n3 = -0.5f * kAsA3,
+                    n4 = -0.5f * kAsA4, n5 = -0.5f * kAsA5;
     constexpr float k_e = -0.72134752044448170f;  // -log2(e) / 2
-    const float ah = fabsf(h);
-    const float t = rcp_approx(fmaf(p_h, ah, 1.0f));
-    const float half_c = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, b5, b4), b3), b2), b1) *
-                         ex2_approx(h * h * k_e);
-    return fmaf(-ah, half_c, fmaxf(h, 0.0f));
+    const float2 ah = make_float2(fabsf(h.x), fabsf(h.y));
+    const float2 den = __ffma2_rn(splat2(p_h), ah, splat2(1.0f));
+    const float2 t = make_float2(rcp_approx(den.x), rcp_approx(den.y));
+    float2 q = __ffma2_rn(t, splat2(n5), splat2(n4));
+    q = __ffma2_rn(t, q, splat2(n3));
+    q = __ffma2_rn(t, q, splat2(n2));
+    q = __ffma2_rn(t, q, splat2(n1));
+    q = __fmul2_rn(t, q);  // -erfc(|h|/sqrt 2) / 2 before the exponential
+    const float2 arg = __fmul2_rn(__fmul2_rn(h, h), splat2(k_e));
+    const float2 neg_half_c = __fmul2_rn(q, make_float2(ex2_approx(arg.x), ex2_approx(arg.y)));
+    return __ffma2_rn(ah, neg_half_c, make_float2(fmaxf(h.x, 0.0f), fmaxf(h.y, 0.0f)));
 }
 
-// Scales 32 fp32 accumulator values by alpha, applies the activation (kGelu)
-// and rounds to 16 packed bf16x2.
+// Scales 32 fp32 accumulator values by alpha (packed pairs), applies the
+// activation (kGelu) and rounds to 16 packed bf16x2.
 template <bool kGelu>
 __device__ __forceinline__ void cvt_32(const uint32_t (&r)[32], float alpha, uint32_t *pk) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-        float h0 = __fmul_rn(__uint_as_float(r[2 * i]), alpha);
-        float h1 = __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha);
-        if (kGelu) {
-            h0 = gelu_erf(h0);
-            h1 = gelu_erf(h1);
-        }
-        const __nv_bfloat162 h = __floats2bfloat162_rn(h0, h1);
-        pk[i] = *reinterpret_cast<const uint32_t *>(&h);
+        float2 h = __fmul2_rn(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
+                              splat2(alpha));
+        if (kGelu) h = gelu_erf2(h);
+        const __nv_bfloat162 b = __floats2bfloat162_rn(h.x, h.y);
+        pk[i] = *reinterpret_cast<const uint32_t *>(&b);
     }
 }
 

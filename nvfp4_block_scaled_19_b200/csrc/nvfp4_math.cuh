@@ -171,11 +171,14 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // E2M1 codes of 8 bf16 values times inv.
+// (The products are packed f32x2 multiplies, each half rounded as __fmul_rn.)
 __device__ __forceinline__ uint32_t quantize_bf16x8(uint4 v, float inv) {
-    return e2m1x8(__fmul_rn(bf16_lo(v.x), inv), __fmul_rn(bf16_hi(v.x), inv),
-                  __fmul_rn(bf16_lo(v.y), inv), __fmul_rn(bf16_hi(v.y), inv),
-                  __fmul_rn(bf16_lo(v.z), inv), __fmul_rn(bf16_hi(v.z), inv),
-                  __fmul_rn(bf16_lo(v.w), inv), __fmul_rn(bf16_hi(v.w), inv));
+    const float2 i2 = make_float2(inv, inv);
+    const float2 p0 = __fmul2_rn(make_float2(bf16_lo(v.x), bf16_hi(v.x)), i2);
+    const float2 p1 = __fmul2_rn(make_float2(bf16_lo(v.y), bf16_hi(v.y)), i2);
+    const float2 p2 = __fmul2_rn(make_float2(bf16_lo(v.z), bf16_hi(v.z)), i2);
+    const float2 p3 = __fmul2_rn(make_float2(bf16_lo(v.w), bf16_hi(v.w)), i2);
+    return e2m1x8(p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y);
 }
 
 // Byte offset of the block scale (row r, block c) in the 128x4-tiled layout

@@ -17,10 +17,8 @@ SRC = Path(__file__).resolve().parents[1] / "nvfp4_block_scaled_19_b200" / "csrc
 
 def _coefficients():
     text = SRC.read_text()
-    body = text[text.index("__device__ __forceinline__ float gelu_erf"):]
-    body = body[:body.index("}")]
-    vals = dict(re.findall(r"(p|a[1-5]) = (-?[0-9.]+)f", body))
-    return {k: float(v) for k, v in vals.items()}
+    vals = dict(re.findall(r"kAs(P|A[1-5]) = (-?[0-9.]+)f", text))
+    return {k.lower(): float(v) for k, v in vals.items()}
 
 
 def _erf_as(x, c):
