@@ -11,9 +11,12 @@ calibrated once from an untimed pass.  The headline metric is NVFP4 GEMM
 TFLOP/s including the activation quantize, i.e. 2*M*N*K / (t_quantize +
 t_gemm) summed over layers.
 
-Multi-GPU: one process per GPU (torchrun); each rank runs an independent
-replica of the workload (the linear layer needs no exchange), so scaling is
-weak and the value is the work of all ranks over the max-over-ranks time.
+Multi-GPU: one process per GPU (torchrun).  By default each rank runs an
+independent replica of the workload (the linear layer needs no exchange), so
+scaling is weak and the value is the work of all ranks over the max-over-
+ranks time.  --shard tokens splits the workload's tokens across the ranks
+instead (strong scaling); the one exchange is an all-reduce(MAX) of each
+layer input's amax, so every row is quantized as on one GPU.
 
 --impl reference times the CPU oracle (test infrastructure, the only
 reference for this path) on a bounded sample of the same workload.
@@ -228,8 +231,12 @@ class ClockSampler:
 
 class Layer:
     def __init__(self, nv, spec, M, x_cpu, w_cpu, device, row_scales=False, fp8=False,
-                 stale=False):
+                 stale=False, m_global=None, sharded=False):
         self.spec = spec
+        # Token shards: this rank's M of the workload's m_global rows; its
+        # drawn input is quantized with the group's amax (one all-reduce).
+        self.m_global = M if m_global is None else m_global
+        self.sharded = sharded and not spec.x_from_prev
         self.row_scales = row_scales
         self.fp8 = fp8
         # One-pass quantize with the previous call's amax: two amax words,
@@ -322,6 +329,9 @@ def run_step(nv, layers, ev=None):
             nv.quantize_fp8(L.x, L.amax, L.xq)
         elif L.row_scales:
             nv.quantize_rowwise(L.x, L.xq)
+        elif L.sharded:
+            from nvfp4_block_scaled_19_b200 import sharded
+            sharded.quantize_sharded(L.x, L.xq, L.amax)
         elif L.stale:
             k = L.calls & 1
             nv.quantize_one_pass(L.x, L.amax_pair[k], L.amax_pair[1 - k], L.xq)
@@ -344,6 +354,9 @@ def calibrate(nv, layers) -> None:
     run_step(nv, layers)
     for L in layers:
         if L.fused is not None:
+            if L.m_global != L.M:   # token shards: one static output scale for the group
+                from nvfp4_block_scaled_19_b200 import sharded
+                sharded.all_reduce_max(L.fused.amax)
             a = L.fused.amax.clamp_min(torch.finfo(torch.float32).tiny)
             L.fused.s_enc.copy_(torch.full_like(a, 2688.0) / a)
     torch.cuda.synchronize()
@@ -353,6 +366,9 @@ def graph_timing(nv, layers, flush, steps, dist, device, world) -> dict:
     """The same step captured once in a CUDA graph and replayed (no host
     launch overhead between the kernels); L2 flushed before every replay,
     outside the timed span."""
+    if world > 1 and any(L.sharded for L in layers):
+        return {"value": None, "note": "not captured: the token-sharded step holds an NCCL "
+                                       "all-reduce"}
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     g = torch.cuda.CUDAGraph()
@@ -378,15 +394,24 @@ def graph_timing(nv, layers, flush, steps, dist, device, world) -> dict:
     ms = sum(a.elapsed_time(b) for a, b in ev)
     sec = max_over_ranks(ms / 1e3, dist, device)
     del g
-    flops = sum(L.flops for L in layers) * steps
-    return {"value": round(aggregate(flops, world, sec) / 1e12, 3), "unit": UNIT,
+    flops = job_flops(layers, world) * steps
+    return {"value": round(flops / sec / 1e12, 3), "unit": UNIT,
             "ms_per_step": round(ms / steps, 5), "steps": steps,
             "kernels_per_step": launches_per_step(layers),
             "note": "one CUDA graph per step (captured once), events around each replay"}
 
 
 def launches_per_step(layers) -> int:
-    return sum(1 + (0 if L.spec.x_from_prev else 2 if L.fp8 else 1) for L in layers)
+    return sum(1 + (0 if L.spec.x_from_prev else 2 if (L.fp8 or L.sharded) else 1)
+               for L in layers)
+
+
+def job_flops(layers, world: int) -> int:
+    """FLOPs of one step over the whole job: replicas each run the whole
+    workload; token shards run it once between them."""
+    if any(L.m_global != L.M for L in layers) or any(L.sharded for L in layers):
+        return sum(2 * L.m_global * L.N * L.K for L in layers)
+    return sum(L.flops for L in layers) * world
 
 
 def gpu_arm(args) -> dict | None:
@@ -401,8 +426,18 @@ def gpu_arm(args) -> dict | None:
     row = args.act_scale == "row"
     stale = args.act_scale == "stale"
     fp8 = args.variant == "fp8"
-    layers = [Layer(nv, l, w.M, *layer_inputs(w, i), device, row_scales=row, fp8=fp8, stale=stale)
-              for i, l in enumerate(w.layers)]
+    shard = args.shard == "tokens"
+    if shard and (fp8 or row or stale):
+        raise SystemExit("--shard tokens runs the per-tensor dynamic NVFP4 path only")
+    from nvfp4_block_scaled_19_b200.sharded import shard_rows
+    r0, r1 = shard_rows(w.M, world, rank) if shard else (0, w.M)
+    layers = []
+    for i, l in enumerate(w.layers):
+        x, wt = layer_inputs(w, i)
+        if shard and x is not None:
+            x = x[r0:r1].contiguous()
+        layers.append(Layer(nv, l, r1 - r0, x, wt, device, row_scales=row, fp8=fp8, stale=stale,
+                            m_global=w.M, sharded=shard))
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     torch.cuda.synchronize()
     calibrate(nv, layers)
@@ -442,8 +477,7 @@ def gpu_arm(args) -> dict | None:
     step_ms = [sum(q_ms[i][s] + g_ms[i][s] for i in range(n_l)) for s in range(args.steps)]
     total_s = sum(step_ms) / 1e3
     total_s = max_over_ranks(total_s, dist, device)
-    flops_step = sum(L.flops for L in layers)
-    value = aggregate(flops_step * args.steps, world, total_s) / 1e12
+    value = job_flops(layers, world) * args.steps / total_s / 1e12
 
     # Roofline of the dominant kernel (the GEMM), live CUDA-event durations.
     g_avg = [sum(g) / len(g) for g in g_ms]
@@ -474,7 +508,7 @@ def gpu_arm(args) -> dict | None:
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3),
         "ms_per_step": round(sum(step_ms) / args.steps, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": "strong" if shard else "weak", "vs_baseline": None,
         "dtype": ("fp8 (e4m3, per-tensor fp32 scales, fp32 accumulate, bf16 out)" if fp8 else
                   "nvfp4 (e2m1 x ue4m3 block scales, fp32 accumulate, bf16 out)"),
         "data": "synthetic (seeded DiT-shaped activations and N(0,1/K) weights)",
@@ -490,7 +524,9 @@ def gpu_arm(args) -> dict | None:
                                         else "per tensor, dynamic (amax + nvfp4_fp8_quantize)"
                                         if fp8 else
                                         "per tensor, dynamic (nvfp4_quantize_dynamic)"),
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": (f"tokens x{world} (rows {r0}..{r1 - 1} on rank {rank}; "
+                                   "one all-reduce(MAX) of the amax per layer and step)"
+                                   if shard else f"replicas x{world}")},
         "pct_fp4_peak": {"of_4x_measured_bf16_burst": round(value / world / fp4_peak, 4),
                          "of_nominal_9pf": round(value / world / NOMINAL_FP4_TFLOPS, 4)}
         if not fp8 else
@@ -532,7 +568,7 @@ def host_e2e(nv, layers, args, device, dist, world) -> dict:
     Independent layers go through nvfp4_linear_host; a chain (a layer fed by
     the previous layer's fused output) through the Python API, copying every
     drawn X in and the last layer's Y out."""
-    if any(L.spec.x_from_prev or L.row_scales or L.fp8 or L.stale for L in layers):
+    if any(L.spec.x_from_prev or L.row_scales or L.fp8 or L.stale or L.sharded for L in layers):
         return chain_e2e(nv, layers, args, device, dist, world)
     stream = torch.cuda.current_stream()
     hosts = []
@@ -587,8 +623,8 @@ def chain_e2e(nv, layers, args, device, dist, world) -> dict:
     e1.record()
     torch.cuda.synchronize()
     sec = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, device)
-    flops = sum(L.flops for L in layers) * steps
-    return {"value": round(aggregate(flops, world, sec) / 1e12, 3), "unit": UNIT,
+    flops = job_flops(layers, world) * steps
+    return {"value": round(flops / sec / 1e12, 3), "unit": UNIT,
             "h2d_bytes_per_step": sum(L.M * L.K * 2 for L, _ in xs),
             "d2h_bytes_per_step": sum(L.M * L.N * 2 for L, _ in ys), "steps": steps,
             "api": "Python API (quantize_dynamic / quantize_rowwise / quantize_one_pass / "
@@ -750,6 +786,9 @@ def main(argv=None) -> int:
     ap.add_argument("--act-scale", choices=["tensor", "row", "stale"], default="tensor",
                     help="activation tensor scale: per tensor (the pages' scheme), per token, "
                          "or per tensor from the previous call's amax (one pass)")
+    ap.add_argument("--shard", choices=["replicas", "tokens"], default="replicas",
+                    help="N > 1: independent replicas (weak scaling) or the workload's tokens "
+                         "split across ranks with one amax all-reduce per layer (strong)")
     ap.add_argument("--quantize-sweep", action="store_true",
                     help="instead of the step: quantize throughput over 2^20..2^29 elements")
     ap.add_argument("--sweep-iters", type=int, default=20)

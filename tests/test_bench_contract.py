@@ -51,3 +51,30 @@ def test_gpu_arm_line():
     # ms_per_step is the evented step; value is the work of the step over it
     assert abs(2 * 4608 * 9216 * 3072 / (d["ms_per_step"] * 1e-3) / 1e12 - d["value"]) \
         < 0.01 * d["value"]
+
+
+class _L:
+    def __init__(self, M, N, K, m_global=None, sharded=False):
+        self.M, self.N, self.K = M, N, K
+        self.m_global = M if m_global is None else m_global
+        self.sharded = sharded
+        self.flops = 2 * M * N * K
+
+
+def test_job_flops_replicas_and_shards():
+    import bench
+    rep = [_L(4608, 9216, 3072)]
+    assert bench.job_flops(rep, 4) == 4 * 2 * 4608 * 9216 * 3072
+    shards = [_L(1152, 9216, 3072, m_global=4608, sharded=True)]
+    assert bench.job_flops(shards, 4) == 2 * 4608 * 9216 * 3072
+    one = [_L(4608, 9216, 3072, m_global=4608, sharded=True)]
+    assert bench.job_flops(one, 1) == 2 * 4608 * 9216 * 3072
+
+
+@pytest.mark.gpu
+def test_gpu_arm_token_shards_one_rank():
+    d = _run(["--shard", "tokens", "--steps", "10", "--warmup", "3", "--no-cpu-baseline",
+              "--e2e-steps", "2"], 600)
+    assert d["scaling"] == "strong" and d["config"]["parallelism"].startswith("tokens x1")
+    assert d["gpu_launches"] == 3 * 10      # amax + quantize + GEMM per step
+    assert d["value"] > 0 and d["e2e"]["value"] > 0

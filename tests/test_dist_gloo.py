@@ -34,7 +34,7 @@ def _worker(rank, world, port, out):
 def test_two_rank_timing_and_aggregation():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     for r in range(world):
@@ -84,3 +84,67 @@ def test_cpu_baseline_sample_is_bounded():
     cb = bench.cpu_baseline(WORKLOADS["tiny_linear"], 0.3)
     assert bench.time.perf_counter() - t0 < 30
     assert cb["seconds"] >= 0.3 and cb["value"] > 0 and "passes of" in cb["sample"]
+
+
+def _shard_worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import numpy as np
+    import torch.distributed as dist
+
+    import oracle
+    from nvfp4_block_scaled_19_b200.sharded import all_reduce_max, shard_rows
+    from workloads import bf16_bits, draw_x
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    M, K = 301, 256
+    x = draw_x("lognormal_channels", M, K, seed=7, index=0)
+    s, e = shard_rows(M, world, rank)
+    xb = bf16_bits(x[s:e])
+    amax = torch.tensor([float(oracle.tensor_amax(xb))], dtype=torch.float32)
+    all_reduce_max(amax)
+    q, sf = oracle.quantize(xb, e - s, K, oracle.tensor_scale(np.float32(amax.item())))
+    out[rank] = (s, e, float(amax.item()), q, sf)
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(180)
+def test_token_shards_quantize_like_one_tensor():
+    """Two gloo ranks each take a slice of the tokens, reduce their amax with
+    the package's all-reduce(MAX) and quantize their rows (with the oracle):
+    every row's codes and block scales are those of the whole tensor's
+    quantization, and the reduced amax is the whole tensor's."""
+    import numpy as np
+
+    import oracle
+    from workloads import bf16_bits, draw_x
+    world = 2
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.spawn(_shard_worker, args=(world, port, out), nprocs=world, join=True)
+    M, K = 301, 256
+    kb = K // 16
+    x = draw_x("lognormal_channels", M, K, seed=7, index=0)
+    fq, fsf, _, famax = oracle.quantize_dynamic(bf16_bits(x), M, K)
+    covered = 0
+    for r in range(world):
+        s, e, amax, q, sf = out[r]
+        assert np.float32(amax) == famax
+        assert np.array_equal(q, fq[s:e])
+        for row in range(s, e):
+            for c in range(kb):
+                assert sf[oracle.sf_offset(row - s, c, kb)] == fsf[oracle.sf_offset(row, c, kb)]
+        covered += e - s
+    assert covered == M
+
+
+def test_shard_rows_partition():
+    from nvfp4_block_scaled_19_b200.sharded import shard_rows
+    for rows in (0, 1, 7, 4608, 16897):
+        for world in (1, 2, 3, 8):
+            spans = [shard_rows(rows, world, r) for r in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == rows
+            assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+            sizes = [e - s for s, e in spans]
+            assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        shard_rows(10, 2, 2)
