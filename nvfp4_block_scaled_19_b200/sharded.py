@@ -29,8 +29,8 @@ def shard_rows(rows: int, world: int, rank: int) -> tuple[int, int]:
 
 def all_reduce_max(t: torch.Tensor, group=None) -> torch.Tensor:
     """In-place MAX over the ranks of `group` (the default group if None);
-    nothing to do without an initialised group of more than one rank."""
-    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+    nothing to do when no process group is initialised (a single process)."""
+    if dist.is_available() and dist.is_initialized():
         dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
     return t
 
