@@ -78,3 +78,15 @@ def test_gpu_arm_token_shards_one_rank():
     assert d["scaling"] == "strong" and d["config"]["parallelism"].startswith("tokens x1")
     assert d["gpu_launches"] == 3 * 10      # amax + quantize + GEMM per step
     assert d["value"] > 0 and d["e2e"]["value"] > 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("mode,launches", [(["--act-scale", "stale"], 2), (["--act-scale", "row"], 2),
+                                           (["--variant", "fp8"], 3)])
+def test_gpu_arm_variants(mode, launches):
+    """The one-pass stale-scale, per-token and FP8 modes print the same line
+    (launches per step: quantize kernels + GEMM)."""
+    d = _run(mode + ["--steps", "5", "--warmup", "3", "--no-cpu-baseline", "--e2e-steps", "2"], 600)
+    assert BASE_KEYS <= set(d)
+    assert d["value"] > 0 and d["gpu_launches"] == launches * 5
+    assert d["roofline"]["frac"] > 0 and d["e2e"]["value"] > 0
