@@ -42,7 +42,7 @@ from workloads import WORKLOADS, layer_inputs  # noqa: E402
 
 METRIC = "NVFP4 GEMM TFLOPS incl. act quantize (% FP4 peak); quantize GB/s (% HBM)"
 UNIT = "TFLOP/s"
-DEFAULT_WORKLOAD = "qkv_1024"
+DEFAULT_WORKLOAD = "ffn_2048"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_PER_BF16 = 4.0      # nominal dense FP4 / dense BF16 (9 / 2.25 PFLOP/s)
@@ -90,11 +90,20 @@ def gemm_source_hash() -> str:
     return h.hexdigest()
 
 
-def profiled_traffic(workload: str) -> tuple[float | None, str]:
-    """DRAM bytes per launch of the workload's dominant GEMM from the committed
-    ncu summary profiles/gemm_pair_<workload>.md, or None when there is none or
-    the kernel sources changed after the capture."""
-    path = os.path.join(ROOT, "profiles", f"gemm_pair_{workload}.md")
+def profile_name(w, layer) -> str:
+    """Name under which a layer's GEMM capture is filed in profiles/: the
+    single-layer workload the layer's tensors come from, else the workload
+    (with the layer's name when the workload has several layers)."""
+    if layer.source is not None:
+        return layer.source[0]
+    return w.name if len(w.layers) == 1 else f"{w.name}_{layer.name}"
+
+
+def profiled_traffic(name: str) -> tuple[float | None, str]:
+    """DRAM bytes per launch of a GEMM from the committed ncu summary
+    profiles/gemm_pair_<name>.md, or None when there is none or the kernel
+    sources changed after the capture."""
+    path = os.path.join(ROOT, "profiles", f"gemm_pair_{name}.md")
     try:
         with open(path) as f:
             kv = dict(l.split(":", 1) for l in f.read().splitlines()
@@ -451,18 +460,13 @@ def gpu_arm(args) -> dict | None:
         raise RuntimeError(f"device wait timed out during warm-up (tag {detail})")
 
     n_l = len(layers)
-    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_l)]
-          for _ in range(args.steps)]
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
     barrier(dist, device)
     torch.cuda.synchronize()
     t_wall0 = time.time()
-    for s in range(args.steps):
-        flush.zero_()          # L2 flush between steps, outside the timed spans
-        run_step(nv, layers, ev[s])
-    torch.cuda.synchronize()
+    q_ms, g_ms = timed_steps(nv, layers, flush, args.steps)
     t_wall1 = time.time()
     barrier(dist, device)
     time.sleep(0.1)
@@ -472,8 +476,6 @@ def gpu_arm(args) -> dict | None:
     if code != 0:
         raise RuntimeError(f"device wait timed out (tag {detail})")
 
-    q_ms = [[ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(args.steps)] for i in range(n_l)]
-    g_ms = [[ev[s][i][1].elapsed_time(ev[s][i][2]) for s in range(args.steps)] for i in range(n_l)]
     step_ms = [sum(q_ms[i][s] + g_ms[i][s] for i in range(n_l)) for s in range(args.steps)]
     total_s = sum(step_ms) / 1e3
     total_s = max_over_ranks(total_s, dist, device)
@@ -494,7 +496,20 @@ def gpu_arm(args) -> dict | None:
     q_gbs = q_bytes / (q_ms_sum * 1e-3) / 1e9 if q_bytes else 0.0
 
     traffic, traffic_src = ((None, "no ncu summary for the FP8 variant") if fp8
-                            else profiled_traffic(w.name))
+                            else profiled_traffic(profile_name(w, layers[top].spec)))
+    per_layer = []
+    for i, L in enumerate(layers):
+        g_tf = L.flops / (g_avg[i] * 1e-3) / 1e12
+        incl = L.flops / ((g_avg[i] + q_avg[i]) * 1e-3) / 1e12
+        per_layer.append({
+            "layer": L.spec.name, "M": L.M, "N": L.N, "K": L.K,
+            "quantize_us": round(q_avg[i] * 1e3, 2), "gemm_us": round(g_avg[i] * 1e3, 2),
+            "gemm_tflops": round(g_tf, 1), "gemm_frac": round(g_tf / fp4_peak, 4),
+            "tflops_incl_quantize": round(incl, 1),
+            "frac_incl_quantize": round(incl / fp4_peak, 4),
+            "fused_output": L.fused is not None})
+    modes = (ffn_down_modes(nv, args, flush, device, fp4_peak)
+             if w.name == "ffn_2048" and not (fp8 or row or stale or shard) else None)
     graph = graph_timing(nv, layers, flush, args.steps, dist, device, world)
     code, detail = nv.device_error()
     if code != 0:
@@ -543,6 +558,7 @@ def gpu_arm(args) -> dict | None:
                               "shared memory where a slice per SM fits, else from L2)")},
         "gemm": {"tflops": round(gemm_tflops, 1), "ms": round(g_avg[top], 5),
                  "layer": layers[top].spec.name},
+        "per_layer": per_layer,
         "roofline": {"bound": "tensor",
                      "kernel": ("gemm_pair_kernel FP8 (tcgen05.mma cta_group::2 kind::f8f6f4)"
                                 if fp8 else gemm_kernel_name(layers[top].M, layers[top].N)),
@@ -558,9 +574,79 @@ def gpu_arm(args) -> dict | None:
         "e2e": e2e,
         "gpu_launches": launches_per_step(layers) * args.steps,
     }
+    if modes is not None:
+        line["ffn_down_modes"] = modes
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     return line
+
+
+def timed_steps(nv, layers, flush, steps):
+    """`steps` passes of the step with the L2 flushed before each, outside the
+    timed spans; per layer the CUDA-event durations (ms) of its quantize and
+    its GEMM in every step."""
+    n_l = len(layers)
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_l)]
+          for _ in range(steps)]
+    for s in range(steps):
+        flush.zero_()          # L2 flush between steps, outside the timed spans
+        run_step(nv, layers, ev[s])
+    torch.cuda.synchronize()
+    q_ms = [[ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(steps)] for i in range(n_l)]
+    g_ms = [[ev[s][i][1].elapsed_time(ev[s][i][2]) for s in range(steps)] for i in range(n_l)]
+    return q_ms, g_ms
+
+
+def ffn_down_modes(nv, args, flush, device, fp4_peak) -> dict:
+    """The FFN down-projection at 2048^2 (M=16896, K=12288, N=3072) in the
+    three ways its input can be produced, each timed like the step (L2 flushed
+    before every pass, CUDA events, `steps` passes):
+      dynamic: amax + quantize of the bf16 input in one launch, then the GEMM
+        (the headline step's second layer, timed here again on its own);
+      stale_scale: one pass over the input with the previous call's amax;
+      fused_producer: the input's codes come straight from the up-projection's
+        epilogue (GELU + NVFP4 quantize), so the down-projection has no
+        quantize of its own; reported for the down GEMM and for the whole FFN
+        block (up-projection with its input quantize, then down)."""
+    def run(wname, stale):
+        w = WORKLOADS[wname]
+        layers = []
+        for i, l in enumerate(w.layers):
+            x, wt = layer_inputs(w, i)
+            layers.append(Layer(nv, l, w.M, x, wt, device, stale=stale))
+        calibrate(nv, layers)
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            run_step(nv, layers)
+        q, g = timed_steps(nv, layers, flush, args.steps)
+        code, detail = nv.device_error()
+        if code != 0:
+            raise RuntimeError(f"device wait timed out (tag {detail})")
+        out = [(L.flops, L.quant_bytes, sum(q[i]) / len(q[i]), sum(g[i]) / len(g[i]))
+               for i, L in enumerate(layers)]
+        del layers
+        torch.cuda.empty_cache()
+        return out
+
+    res = {}
+    for name, stale in (("dynamic", False), ("stale_scale", True)):
+        (fl, qb, q, g), = run("ffn_down_2048", stale)
+        res[name] = {"quantize_us": round(q * 1e3, 2), "gemm_us": round(g * 1e3, 2),
+                     "tflops_incl_quantize": round(fl / ((q + g) * 1e-3) / 1e12, 1),
+                     "frac_incl_quantize": round(fl / ((q + g) * 1e-3) / 1e12 / fp4_peak, 4),
+                     "quantize_gbs": round(qb / (q * 1e-3) / 1e9, 1)}
+    (fu, _, qu, gu), (fd, _, _, gd) = run("ffn_block_2048", False)
+    flops = fu + fd
+    res["fused_producer"] = {
+        "down_gemm_us": round(gd * 1e3, 2),
+        "down_tflops": round(fd / (gd * 1e-3) / 1e12, 1),
+        "up_quantize_us": round(qu * 1e3, 2), "up_gemm_gelu_quantize_us": round(gu * 1e3, 2),
+        "block_tflops_incl_quantize": round(flops / ((qu + gu + gd) * 1e-3) / 1e12, 1),
+        "block_frac_incl_quantize": round(flops / ((qu + gu + gd) * 1e-3) / 1e12 / fp4_peak, 4),
+        "note": "ffn_block_2048: the up-projection's epilogue applies GELU and writes the "
+                "down-projection's NVFP4 codes and scales (static scale calibrated once)"}
+    res["peak_tflops"] = round(fp4_peak, 1)
+    return res
 
 
 def host_e2e(nv, layers, args, device, dist, world) -> dict:

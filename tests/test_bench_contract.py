@@ -25,7 +25,7 @@ def test_reference_arm_line():
     d = _run(["--impl", "reference", "--steps", "2", "--warmup", "1", "--cpu-seconds", "0.5"], 300)
     assert BASE_KEYS <= set(d)
     assert d["impl"] == "reference" and d["steps"] == 2 and d["n_gpus"] == 1
-    assert d["config"]["workload"] == "qkv_1024" and d["value"] > 0
+    assert d["config"]["workload"] == "ffn_2048" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
@@ -38,19 +38,33 @@ def test_gpu_arm_line():
     assert BASE_KEYS <= set(d)
     assert d["n_gpus"] == 1 and d["steps"] == 20 and d["warmup"] == 3
     assert d["higher_is_better"] is True and d["scaling"] == "weak"
-    assert d["config"]["workload"] == "qkv_1024"
+    # The default step: the 2048^2 FFN GEMMs (up, then down with the fused
+    # next-layer quantize), each with the dynamic quantize of its input.
+    assert d["config"]["workload"] == "ffn_2048"
+    M, H, F = 16896, 3072, 12288
     r = d["roofline"]
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert 0 < r["frac"] < 1.5 and abs(r["achieved"] / r["peak"] - r["frac"]) < 1e-3
     assert r["traffic"] is None or r["traffic"] > 0
     e = d["e2e"]
-    assert e["h2d_bytes_per_step"] == 4608 * 3072 * 2 and e["d2h_bytes_per_step"] == 4608 * 9216 * 2
+    assert e["h2d_bytes_per_step"] == 2 * M * (H + F)
+    assert e["d2h_bytes_per_step"] == 2 * M * (F + H)
     assert 0 < e["value"] < d["value"]
-    assert d["gpu_launches"] == 2 * 20
+    assert d["gpu_launches"] == 4 * 20
     assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(d["clocks"])
     # ms_per_step is the evented step; value is the work of the step over it
-    assert abs(2 * 4608 * 9216 * 3072 / (d["ms_per_step"] * 1e-3) / 1e12 - d["value"]) \
-        < 0.01 * d["value"]
+    flops = 2 * M * F * H * 2
+    assert abs(flops / (d["ms_per_step"] * 1e-3) / 1e12 - d["value"]) < 0.01 * d["value"]
+    pl = d["per_layer"]
+    assert [p["layer"] for p in pl] == ["ffn_up", "ffn_down"]
+    assert abs(sum(p["quantize_us"] + p["gemm_us"] for p in pl) - d["ms_per_step"] * 1e3) \
+        < 0.01 * d["ms_per_step"] * 1e3
+    for p in pl:
+        assert 0 < p["gemm_frac"] < 1.5 and p["tflops_incl_quantize"] < p["gemm_tflops"]
+    m = d["ffn_down_modes"]
+    assert {"dynamic", "stale_scale", "fused_producer"} <= set(m)
+    assert m["stale_scale"]["quantize_us"] < m["dynamic"]["quantize_us"]
+    assert m["fused_producer"]["block_tflops_incl_quantize"] > 0
 
 
 class _L:
@@ -73,8 +87,8 @@ def test_job_flops_replicas_and_shards():
 
 @pytest.mark.gpu
 def test_gpu_arm_token_shards_one_rank():
-    d = _run(["--shard", "tokens", "--steps", "10", "--warmup", "3", "--no-cpu-baseline",
-              "--e2e-steps", "2"], 600)
+    d = _run(["--workload", "qkv_1024", "--shard", "tokens", "--steps", "10", "--warmup", "3",
+              "--no-cpu-baseline", "--e2e-steps", "2"], 600)
     assert d["scaling"] == "strong" and d["config"]["parallelism"].startswith("tokens x1")
     assert d["gpu_launches"] == 3 * 10      # amax + quantize + GEMM per step
     assert d["value"] > 0 and d["e2e"]["value"] > 0
@@ -86,7 +100,8 @@ def test_gpu_arm_token_shards_one_rank():
 def test_gpu_arm_variants(mode, launches):
     """The one-pass stale-scale, per-token and FP8 modes print the same line
     (launches per step: quantize kernels + GEMM)."""
-    d = _run(mode + ["--steps", "5", "--warmup", "3", "--no-cpu-baseline", "--e2e-steps", "2"], 600)
+    d = _run(mode + ["--workload", "qkv_1024", "--steps", "5", "--warmup", "3",
+                     "--no-cpu-baseline", "--e2e-steps", "2"], 600)
     assert BASE_KEYS <= set(d)
     assert d["value"] > 0 and d["gpu_launches"] == launches * 5
     assert d["roofline"]["frac"] > 0 and d["e2e"]["value"] > 0

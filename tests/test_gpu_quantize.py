@@ -5,7 +5,7 @@ import torch
 
 from gpu_common import (assert_quant_equal, gpu_quantize_dynamic, oracle_quantize_dynamic,
                         require_cuda)
-from workloads import WORKLOADS, bf16_bits, draw_x, layer_inputs
+from workloads import OWN_WORKLOADS, WORKLOADS, bf16_bits, draw_x, layer_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -122,7 +122,7 @@ def test_quantize_static_scale(nv, orc):
         assert np.float32(t.s_dec.item()) == orc.decode_scale(np.float32(s))
 
 
-@pytest.mark.parametrize("name", list(WORKLOADS))
+@pytest.mark.parametrize("name", OWN_WORKLOADS)
 def test_quantize_workloads_full_size(nv, name):
     """Activations (per-call, single-launch path) and weights (load-time,
     two-kernel path) of every workload, at full size, bit-exact."""

@@ -39,6 +39,10 @@ class Layer:
     act: str = "none"        # activation of a fused epilogue: "none" | "gelu"
     x_from_prev: bool = False  # X is the previous layer's fused NVFP4 output (not drawn)
     keep_y: bool = True      # the bf16 Y is needed (False: only the fused output)
+    # Draw X and W exactly as layer `source[1]` of workload `source[0]` does
+    # (same seed and generator indices), so a step that strings together the
+    # layers of several single-layer workloads times the same tensors.
+    source: tuple[str, int] | None = None
 
 
 @dataclass(frozen=True)
@@ -78,6 +82,17 @@ WORKLOADS: dict[str, Workload] = {
         "output feeds a fused next-layer NVFP4 quantize",
         M=16896, seed=3,
         layers=(Layer("ffn_down", K=12288, N=3072, x_dist="gelu", w_std=None, fused_out=True),)),
+    "ffn_2048": Workload(
+        "ffn_2048",
+        "The DiT FFN GEMMs at 2048^2, each with the dynamic NVFP4 quantize of its input: "
+        "up-projection M=16896, K=3072, N=12288, then down-projection M=16896, K=12288, "
+        "N=3072 whose output feeds a fused next-layer NVFP4 quantize (inputs drawn as in "
+        "ffn_up_2048 and ffn_down_2048)",
+        M=16896, seed=2,
+        layers=(Layer("ffn_up", K=3072, N=12288, x_dist="lognormal_channels", w_std=None,
+                      source=("ffn_up_2048", 0)),
+                Layer("ffn_down", K=12288, N=3072, x_dist="gelu", w_std=None, fused_out=True,
+                      source=("ffn_down_2048", 0)))),
     "block_chain_2048": Workload(
         "block_chain_2048",
         "Full DiT block linear chain, CFG batch 2 at 2048^2: M=33792 through QKV "
@@ -97,6 +112,10 @@ WORKLOADS: dict[str, Workload] = {
                 Layer("ffn_down", K=12288, N=3072, x_dist="gelu", w_std=None,
                       x_from_prev=True))),
 }
+
+
+# Workloads that draw tensors of their own (not only layers of other workloads).
+OWN_WORKLOADS = [n for n, w in WORKLOADS.items() if not all(l.source for l in w.layers)]
 
 
 def _gen(seed: int, index: int) -> torch.Generator:
@@ -139,9 +158,12 @@ def layer_inputs(w: Workload, li: int, M: int | None = None):
     tests.  X is None for a layer whose input is the previous layer's fused
     output."""
     l = w.layers[li]
+    seed = w.seed
+    if l.source is not None:
+        seed, li = WORKLOADS[l.source[0]].seed, l.source[1]
     m = w.M if M is None else M
-    x = None if l.x_from_prev else draw_x(l.x_dist, m, l.K, w.seed, index=10 * li)
-    wt = draw_w(l.N, l.K, l.w_std, w.seed, index=10 * li + 1)
+    x = None if l.x_from_prev else draw_x(l.x_dist, m, l.K, seed, index=10 * li)
+    wt = draw_w(l.N, l.K, l.w_std, seed, index=10 * li + 1)
     return x, wt
 
 
