@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.nvfp4_quantize_dynamic_workspace_bytes.argtypes = []
         L.nvfp4_quantize_dynamic.restype = st
         L.nvfp4_quantize_dynamic.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp, vp]
+        L.nvfp4_quantize_dynamic_noalloc.restype = st
+        L.nvfp4_quantize_dynamic_noalloc.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
         L.nvfp4_gemm.restype = st
         L.nvfp4_gemm.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp,
                                  ctypes.POINTER(FusedOut), vp]
@@ -368,12 +370,15 @@ class NVFP4Linear:
         return gemm(xq, self.w, y, fused, want_y)
 
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, ws: dict,
-                     stream=None) -> None:
-        """Host bf16 X -> host bf16 Y through nvfp4_linear_host (copies included)."""
+                     stream=None, single_launch: bool = True) -> None:
+        """Host bf16 X -> host bf16 Y through nvfp4_linear_host (copies included).
+        single_launch=False passes no dynamic-quantize workspace, so the call
+        quantizes X with nvfp4_tensor_amax + nvfp4_quantize."""
         M = x_host.shape[0]
         w = LinearWorkspace(ws["x"].data_ptr(), ws["xq"].data_ptr(), ws["xsf"].data_ptr(),
                             ws["amax"].data_ptr(), ws["s_dec"].data_ptr(), ws["y"].data_ptr(),
-                            dynamic_workspace(ws["x"].device).data_ptr())
+                            dynamic_workspace(ws["x"].device).data_ptr() if single_launch
+                            else None)
         _check("nvfp4_linear_host", lib().nvfp4_linear_host(
             x_host.data_ptr(), M, self.K, self.w.q.data_ptr(), self.w.sf.data_ptr(),
             self.w.s_dec.data_ptr(), self.N, y_host.data_ptr(), ctypes.byref(w),

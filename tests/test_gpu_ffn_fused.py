@@ -9,14 +9,15 @@ fp64, applies its own GELU, rounds to bf16 and quantizes.  The GPU's bf16 Y
 must lie within the GEMM tolerance carried through GELU (whose slope is at
 most 1.129, at h = sqrt 2); every 16-element block whose bf16 values equal
 the oracle's must carry the oracle's codes and scale, and the others (a value
-rounded the other way after a different fp32 summation order) must
-dequantize within the NVFP4 error bound."""
+rounded the other way after a different fp32 summation order) must carry the
+oracle's scale code or, when their largest magnitude differs, a neighbouring
+one, and decode to within one scale unit of the GPU's own values."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from gpu_common import TOL, bf16_from_fp64, require_cuda
+from gpu_common import TOL, bf16_from_fp64, check_fused_blocks, require_cuda
 from workloads import WORKLOADS, bf16_bits, draw_w, draw_x, layer_inputs
 
 pytestmark = pytest.mark.gpu
@@ -64,39 +65,6 @@ def _check_gelu_y(yg, ref_pre, what):
     return g
 
 
-def _decode_block(orc, sf_code, qbytes, s_dec):
-    codes = np.stack([qbytes & 0xF, qbytes >> 4], -1).reshape(-1)
-    return np.array([orc.e2m1_value(int(c)) for c in codes]) * orc.e4m3_value(int(sf_code)) * s_dec
-
-
-def _check_fused_blocks(orc, yg, refb, gq, gsf, g_rows, s_enc_y, what):
-    """yg, refb: [R, N] GPU and oracle bf16 values of the rows g_rows of the
-    GPU's output; gq/gsf: the GPU's full fused codes and tiled scales."""
-    R, N = refb.shape
-    kb = N // 16
-    oq, osf = orc.quantize(bf16_bits(torch.from_numpy(refb).to(torch.bfloat16)), R, N,
-                           np.float32(s_enc_y))
-    s_dec = float(np.float32(1.0) / np.float32(s_enc_y))
-    same = other = 0
-    for i, r in enumerate(g_rows):
-        eq = (yg[i] == refb[i]).reshape(kb, 16).all(axis=1)
-        for c in range(kb):
-            gs = gsf[orc.sf_offset(int(r), c, kb)]
-            gqb = gq[r, c * 8:(c + 1) * 8]
-            if eq[c]:
-                same += 1
-                assert gs == osf[orc.sf_offset(i, c, kb)], (what, r, c)
-                assert np.array_equal(gqb, oq[i, c * 8:(c + 1) * 8]), (what, r, c)
-            else:
-                other += 1
-                deq = _decode_block(orc, gs, gqb, s_dec)
-                blk = refb[i, c * 16:(c + 1) * 16]
-                bound = orc.e4m3_value(int(gs)) * s_dec * 1.01 + 2 * TOL * np.abs(blk).max()
-                assert np.all(np.abs(deq - blk) <= bound), (what, r, c)
-    assert same > 0.8 * (same + other), f"{what}: only {same} of {same + other} blocks equal"
-    return oq, osf
-
-
 SHAPES = [(256, 256, 64), (130, 208, 128), (128, 512, 256), (300, 512, 576), (64, 1024, 3072)]
 
 
@@ -118,7 +86,7 @@ def test_fused_gelu_quantize(nv, orc, M, N, K):
     g = _check_gelu_y(yg, ref_pre, f"{M}x{N}x{K} Y")
     gq = fq.out.q.cpu().numpy()
     gsf = fq.out.sf.cpu().numpy()
-    _, osf = _check_fused_blocks(orc, yg, bf16_from_fp64(g), gq, gsf, np.arange(M), s_enc_y,
+    _, osf = check_fused_blocks(orc, yg, bf16_from_fp64(g), gq, gsf, np.arange(M), s_enc_y,
                                  f"{M}x{N}x{K}")
     kb = N // 16
     pad = [orc.sf_offset(r, c, kb) for r in range(M, (M + 127) // 128 * 128) for c in range(kb)]
@@ -167,7 +135,7 @@ def test_ffn_block_chain_sampled(nv, orc):
     ref_up = _oracle_pre(x, w_up, rows=rows)
     hg = h[rows_t].float().cpu().numpy()
     g = _check_gelu_y(hg, ref_up, "ffn_block up Y")
-    oq, osf = _check_fused_blocks(orc, hg, bf16_from_fp64(g), fq.out.q.cpu().numpy(),
+    oq, osf = check_fused_blocks(orc, hg, bf16_from_fp64(g), fq.out.q.cpu().numpy(),
                                   fq.out.sf.cpu().numpy(), rows, s_enc_h, "ffn_block H")
     # The oracle's own chain: its quantized H (rows only) through the down GEMM.
     s_dec_h = np.float32(1.0) / np.float32(s_enc_h)
