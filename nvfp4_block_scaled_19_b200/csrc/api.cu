@@ -6,9 +6,11 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
+#include "api_checks.h"
 #include "gemm.h"
 #include "nvfp4.h"
 
@@ -20,12 +22,22 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// Per device: the SM count, published by a release store of `state` (0
+// unknown, 1 supported, 2 unsupported), so host threads that make their first
+// calls at the same time read either "unknown" or a complete entry.
 struct DeviceInfo {
-    int state;  // 0 unknown, 1 supported, 2 unsupported
-    int num_sms;
+    std::atomic<int> state;
+    std::atomic<int> num_sms;
 };
 DeviceInfo g_devices[kMaxDevices];
 
+}  // namespace
+
+namespace nvfp4 {
+
+// The library ships one sm_100a image, so only compute capability 10.0 can
+// run its kernels; any other device (other 10.x parts included) is refused
+// up front instead of failing at launch.
 nvfp4_status current_device(int *num_sms) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -33,36 +45,50 @@ nvfp4_status current_device(int *num_sms) {
         return NVFP4_ERR_UNSUPPORTED_DEVICE;
     }
     DeviceInfo &d = g_devices[dev];
-    if (d.state == 0) {
-        int major = 0, sms = 0;
+    int state = d.state.load(std::memory_order_acquire);
+    if (state == 0) {
+        int major = 0, minor = 0, sms = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
             cudaGetLastError();
             return NVFP4_ERR_UNSUPPORTED_DEVICE;
         }
-        d.num_sms = sms;
-        d.state = (major == 10) ? 1 : 2;
+        state = (major == 10 && minor == 0) ? 1 : 2;
+        d.num_sms.store(sms, std::memory_order_relaxed);
+        d.state.store(state, std::memory_order_release);
     }
-    if (d.state != 1) return NVFP4_ERR_UNSUPPORTED_DEVICE;
-    *num_sms = d.num_sms;
+    if (state != 1) return NVFP4_ERR_UNSUPPORTED_DEVICE;
+    *num_sms = d.num_sms.load(std::memory_order_relaxed);
     return NVFP4_OK;
 }
+
+}  // namespace nvfp4
+
+namespace {
+
+using nvfp4::current_device;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 nvfp4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH; }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    // Looked up once; atomic because host threads may make their first calls
+    // at the same time (they all store the same entry point).
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> cached{nullptr};
+    PFN_cuTensorMapEncodeTiled_v12000 fn = cached.load(std::memory_order_acquire);
     if (fn == nullptr) {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
                 cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
+            q == cudaDriverEntryPointSuccess) {
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-        else
+            cached.store(fn, std::memory_order_release);
+        } else {
             cudaGetLastError();
+        }
     }
     return fn;
 }
@@ -117,6 +143,10 @@ bool encode_sf_map(CUtensorMap *m, const void *base, int64_t rows, int64_t K, ui
     return r == CUDA_SUCCESS;
 }
 
+}  // namespace
+
+namespace nvfp4 {
+
 nvfp4_status check_quantize_args(const void *x, int64_t rows, int64_t cols, const void *scale,
                                  const uint8_t *q, const uint8_t *sf) {
     if (rows < 0 || cols <= 0 || cols % 16 != 0) return NVFP4_ERR_INVALID_ARG;
@@ -128,6 +158,12 @@ nvfp4_status check_quantize_args(const void *x, int64_t rows, int64_t cols, cons
     if (!aligned16(x) || !aligned16(q) || !aligned16(sf)) return NVFP4_ERR_MISALIGNED;
     return NVFP4_OK;
 }
+
+}  // namespace nvfp4
+
+namespace {
+
+using nvfp4::check_quantize_args;
 
 nvfp4_status quantize_impl(const void *x, int64_t rows, int64_t cols, const float *scale,
                            bool dynamic, uint8_t *q, uint8_t *sf, float *s_dec_out,

@@ -38,6 +38,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "gemm.h"
@@ -60,15 +61,19 @@ cudaError_t read_and_clear_device_error(int *code, int *detail) {
 }
 
 int *device_error_word() {
-    static int *addr[64] = {nullptr};
+    // Per device, taken once; atomic because host threads may make their
+    // first calls at the same time (they all store the same address).
+    static std::atomic<int *> addr[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (addr[dev] == nullptr) {
-        void *a = nullptr;
-        if (cudaGetSymbolAddress(&a, g_error) != cudaSuccess) return nullptr;
-        addr[dev] = static_cast<int *>(a);
+    int *a = addr[dev].load(std::memory_order_acquire);
+    if (a == nullptr) {
+        void *v = nullptr;
+        if (cudaGetSymbolAddress(&v, g_error) != cudaSuccess) return nullptr;
+        a = static_cast<int *>(v);
+        addr[dev].store(a, std::memory_order_release);
     }
-    return addr[dev];
+    return a;
 }
 
 // Failure-detection self-test: one warp waits, through the kernels' own
@@ -431,15 +436,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 template <class Cfg, bool kGelu>
 static cudaError_t launch_cfg(const GemmMaps &maps, const GemmParams &p, int num_sms,
                               cudaStream_t stream) {
-    static int configured_device = -1;
+    static std::atomic<int> configured[64];
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_device != dev) {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(gemm_kernel<Cfg, kGelu>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        configured_device = dev;
+        configured[dev].store(1, std::memory_order_release);
     }
     const int64_t tiles = ((p.M + kBM - 1) / kBM) * ((p.N + Cfg::BN - 1) / Cfg::BN);
     const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);

@@ -103,10 +103,10 @@ __device__ __forceinline__ void cvt_32(const uint32_t (&r)[32], float alpha, uin
 }
 
 // Reads NC (64 or 128) fp32 accumulator columns of this warp's 32 TMEM lanes
-// (taddr = lane base + first column) into packed bf16x2 (alpha, activation
-// kGelu, rounding).  Two 32-column loads are in flight at a time.
+// (taddr = lane base + first column) into NC / 2 packed bf16x2 at pk (alpha,
+// activation kGelu, rounding).  Two 32-column loads are in flight at a time.
 template <int NC, bool kGelu>
-__device__ __forceinline__ void drain_cols(uint32_t taddr, float alpha, uint32_t (&pk)[NC / 2]) {
+__device__ __forceinline__ void drain_cols(uint32_t taddr, float alpha, uint32_t *pk) {
     static_assert(NC == 64 || NC == 128, "64 or 128 columns");
 #pragma unroll
     for (int ch = 0; ch < NC / 32; ch += 2) {

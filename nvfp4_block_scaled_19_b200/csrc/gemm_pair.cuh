@@ -461,12 +461,14 @@ template <bool kGelu, bool kFp8>
 inline cudaError_t launch_pair(const GemmMaps &maps, const GemmParams &p, int num_sms,
                                cudaStream_t stream) {
     using Cfg = PairCfgFor<kGelu>;
-    static int configured[64] = {0};
-    static int max_clusters[64] = {0};
+    // Per device: clusters that fit at once, published by `configured`
+    // (atomics: host threads may make their first calls concurrently).
+    static std::atomic<int> configured[64];
+    static std::atomic<int> max_clusters[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!configured[dev]) {
+    if (!configured[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(gemm_pair_kernel<Cfg, kGelu, kFp8>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
         if (e != cudaSuccess) return e;
@@ -480,11 +482,11 @@ inline cudaError_t launch_pair(const GemmMaps &maps, const GemmParams &p, int nu
             cudaGetLastError();
             n = num_sms / 2;
         }
-        max_clusters[dev] = n;
-        configured[dev] = 1;
+        max_clusters[dev].store(n, std::memory_order_relaxed);
+        configured[dev].store(1, std::memory_order_release);
     }
     const int64_t tiles = ((p.M + 255) / 256) * ((p.N + 255) / 256);
-    int64_t pairs = max_clusters[dev];
+    int64_t pairs = max_clusters[dev].load(std::memory_order_relaxed);
     if (pairs > tiles) pairs = tiles;
     gemm_pair_kernel<Cfg, kGelu, kFp8><<<static_cast<unsigned>(2 * pairs), Cfg::THREADS,
                                 Cfg::SMEM_BYTES, stream>>>(maps, p);

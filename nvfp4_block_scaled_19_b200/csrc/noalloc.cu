@@ -10,8 +10,10 @@
 // outputs and nothing is allocated, here or in anything it calls.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
+#include "api_checks.h"
 #include "gemm.h"
 #include "nvfp4.h"
 
@@ -22,11 +24,17 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = 256;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
+// A host object whose only use is to be a non-NULL workspace argument of the
+// shared argument check.
+const char g_noalloc_scratch_tag[1] = {0};
+
 static_assert(sizeof(nvfp4::DynWorkspace) <= kNoAllocScratchBytes,
               "the dynamic-quantize workspace must fit the scratch array");
 
 constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices] = {nullptr};
+// Per device, the array's device address once taken (atomic: host threads
+// may make their first calls at the same time; they all store the same value).
+std::atomic<void *> g_scratch_addr[kMaxDevices];
 
 // Device address of the scratch array on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is taken once
@@ -37,15 +45,15 @@ nvfp4_status scratch_address(void **out) {
         cudaGetLastError();
         return NVFP4_ERR_UNSUPPORTED_DEVICE;
     }
-    if (g_scratch_addr[dev] == nullptr) {
-        void *p = nullptr;
+    void *p = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
             cudaGetLastError();
             return NVFP4_ERR_LAUNCH;
         }
-        g_scratch_addr[dev] = p;
+        g_scratch_addr[dev].store(p, std::memory_order_release);
     }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return NVFP4_OK;
 }
 
@@ -55,19 +63,22 @@ extern "C" nvfp4_status nvfp4_quantize_dynamic_noalloc(const void *x_bf16, int64
                                                        int64_t cols, uint8_t *q_out,
                                                        uint8_t *sf_out, float *s_dec_out,
                                                        float *amax_out, nvfp4_stream_t stream) {
-    // Arguments first, so a bad call is refused before any device work.
-    if (rows < 0 || cols <= 0 || cols % 16 != 0 || x_bf16 == nullptr || q_out == nullptr ||
-        sf_out == nullptr)
-        return NVFP4_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(x_bf16) | reinterpret_cast<uintptr_t>(q_out) |
-         reinterpret_cast<uintptr_t>(sf_out)) & 15u)
-        return NVFP4_ERR_MISALIGNED;
+    // The same argument and device checks as nvfp4_quantize_dynamic, done
+    // first, so a call it would refuse is refused here before anything is
+    // enqueued on the shared array (the workspace argument those checks want
+    // non-NULL is this library's own array, so any non-NULL stand-in does).
+    nvfp4_status st = nvfp4::check_quantize_args(x_bf16, rows, cols, g_noalloc_scratch_tag,
+                                                 q_out, sf_out);
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    st = nvfp4::current_device(&sms);
+    if (st != NVFP4_OK) return st;
     // The workspace this call needs does not grow with the tensor; a request
     // for more than the array holds is refused rather than overrunning it.
     if (nvfp4_quantize_dynamic_workspace_bytes() > kNoAllocScratchBytes)
         return NVFP4_ERR_INVALID_ARG;
     void *scratch = nullptr;
-    nvfp4_status st = scratch_address(&scratch);
+    st = scratch_address(&scratch);
     if (st != NVFP4_OK) return st;
     // The array keeps whatever the previous call left; the barrier counter and
     // the amax words must start at zero, so clear them on this stream first.

@@ -30,6 +30,7 @@
 //   row-stream kernel (quantize_rows).
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "gemm.h"
@@ -931,13 +932,17 @@ __global__ void __launch_bounds__(kResThreads, 1) quantize_dynamic_resident_kern
 cudaError_t launch_quantize_dynamic(const void *x, int64_t rows, int64_t cols, uint8_t *q,
                                     uint8_t *sf, float *s_dec_out, float *amax_out,
                                     DynWorkspace *ws, int num_sms, cudaStream_t stream) {
-    static int resident_rows[64] = {0};
-    static int resident_flat[64] = {0};
+    // Per device, from the occupancy queries (atomics: host threads may make
+    // their first calls concurrently; they all store the same values).
+    static std::atomic<int> resident_rows[64];
+    static std::atomic<int> resident_flat[64];
+    static std::atomic<int> res_ready[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     const bool flat = cols % 64 == 0;
-    int &resident = flat ? resident_flat[dev] : resident_rows[dev];
+    std::atomic<int> &resident_slot = flat ? resident_flat[dev] : resident_rows[dev];
+    int resident = resident_slot.load(std::memory_order_relaxed);
     if (resident == 0) {
         int per_sm = 0;
         // Both index widths of the flat kernel have the same launch bounds.
@@ -947,6 +952,7 @@ cudaError_t launch_quantize_dynamic(const void *x, int64_t rows, int64_t cols, u
                                                                  kDynThreads, 0);
         if (e != cudaSuccess || per_sm < 1) return e != cudaSuccess ? e : cudaErrorInvalidValue;
         resident = per_sm;
+        resident_slot.store(per_sm, std::memory_order_relaxed);
     }
     int grid = num_sms * resident;
     int *err = device_error_word();
@@ -969,8 +975,8 @@ cudaError_t launch_quantize_dynamic(const void *x, int64_t rows, int64_t cols, u
         const int64_t per = ((nvec_all + num_sms - 1) / num_sms + 3) / 4 * 4;
         if (per * 32 <= kResMaxBytes && nvec_all < (int64_t(1) << 31) &&
             sf_all < (int64_t(1) << 31)) {
-            static int res_ready[64] = {0};
-            if (!res_ready[dev]) {
+            int ready = res_ready[dev].load(std::memory_order_relaxed);
+            if (ready == 0) {
                 e = cudaFuncSetAttribute(quantize_dynamic_resident_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kResMaxBytes));
@@ -980,9 +986,10 @@ cudaError_t launch_quantize_dynamic(const void *x, int64_t rows, int64_t cols, u
                     &per_sm, quantize_dynamic_resident_kernel, kResThreads,
                     static_cast<size_t>(kResMaxBytes));
                 if (e != cudaSuccess) return e;
-                res_ready[dev] = per_sm >= 1 ? 1 : -1;
+                ready = per_sm >= 1 ? 1 : -1;
+                res_ready[dev].store(ready, std::memory_order_relaxed);
             }
-            if (res_ready[dev] == 1) {
+            if (ready == 1) {
                 cfg.gridDim = dim3(num_sms);
                 cfg.blockDim = dim3(kResThreads);
                 cfg.dynamicSmemBytes = static_cast<size_t>(per * 32);

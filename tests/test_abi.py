@@ -115,3 +115,34 @@ def test_valid_call_without_device_reports_unsupported(L):
     p = _aligned(b)
     assert L.nvfp4_quantize(p, 4, 32, p, p, p, None, None) == 3
     assert L.nvfp4_gemm(p, p, p, p, p, p, 128, 128, 128, p, None, None) == 3
+
+
+def test_noalloc_refuses_exactly_what_quantize_dynamic_refuses(L):
+    """The no-allocation entry point answers every call that the entry point
+    with a caller workspace answers with an argument error the same way, and
+    before anything is enqueued (no device is touched here)."""
+    b = _dev_buf()
+    p = _aligned(b)
+    ws = _aligned(b, 2048)
+    qd, na = L.nvfp4_quantize_dynamic, L.nvfp4_quantize_dynamic_noalloc
+    cases = [
+        (None, 0, 32, None, None),           # empty tensor, NULL arrays: allowed
+        (p, 0, 32, p, p),                    # empty tensor
+        (p, 4, 24, p, p),                    # cols % 16 != 0
+        (p, -1, 32, p, p),                   # negative rows
+        (p, 4, 0, p, p),                     # no columns
+        (p, (1 << 40) // 32 + 1, 32, p, p),  # rows * cols above 2^40
+        (None, 4, 32, p, p),                 # NULL input with rows
+        (p, 4, 32, None, p),                 # NULL codes
+        (p, 4, 32, p, None),                 # NULL scales
+        (p + 2, 4, 32, p, p),                # misaligned input
+        (p, 4, 32, p + 8, p),                # misaligned codes
+        (p, 4, 32, p, p + 4),                # misaligned scales
+        (p, 4, 32, p, p),                    # valid
+    ]
+    for x, rows, cols, q, sf in cases:
+        a = qd(x, rows, cols, q, sf, None, None, ws, None)
+        n = na(x, rows, cols, q, sf, None, None, None)
+        assert a == n, (rows, cols, a, n)
+    assert qd(p, (1 << 40) // 32 + 1, 32, p, p, None, None, ws, None) == 1
+    assert na(p + 2, 4, 32, p, p, None, None, None) == 2
