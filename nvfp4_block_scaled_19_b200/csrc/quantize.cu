@@ -252,8 +252,48 @@ __device__ __forceinline__ bool grid_amax_barrier(DynWorkspace *ws, unsigned gen
     }
 }
 
+// L2 eviction-priority policies for loads (createpolicy): lines loaded with
+// evict_last stay in L2 ahead of normal and evict_first lines.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// 32 bytes at p (16-byte aligned at least) with an L2 policy, bypassing L1.
+__device__ __forceinline__ BF16x16 ldg_32B_policy(const uint8_t *p, bool aligned32, uint64_t pol) {
+    BF16x16 v;
+    if (aligned32) {
+        asm volatile(
+            "ld.global.nc.L1::no_allocate.L2::cache_hint.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7},"
+            " [%8], %9;"
+            : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]),
+              "=r"(v.w[6]), "=r"(v.w[7])
+            : "l"(p), "l"(pol));
+    } else {
+        asm volatile(
+            "ld.global.nc.L1::no_allocate.L2::cache_hint.v4.b32 {%0, %1, %2, %3}, [%4], %5;"
+            : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3])
+            : "l"(p), "l"(pol));
+        asm volatile(
+            "ld.global.nc.L1::no_allocate.L2::cache_hint.v4.b32 {%0, %1, %2, %3}, [%4], %5;"
+            : "=r"(v.w[4]), "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
+            : "l"(p + 16), "l"(pol));
+    }
+    return v;
+}
+
 constexpr int kFlatThreads = 512;
 constexpr int kFlatU = 4;  // 16-element blocks (32-byte loads) in flight per thread
+// Input bytes the single-launch quantize keeps in L2 between its two passes
+// (of the 126 MB L2, leaving room for the codes and scales it writes).
+constexpr int64_t kFlatKeepBytes = int64_t(80) << 20;
 
 // Flat dynamic quantization for cols % 64 == 0 (so 4 consecutive blocks never
 // straddle a row and the scale layout has no column padding).  Block v of the
@@ -283,15 +323,26 @@ __global__ void __launch_bounds__(kFlatThreads, 2) quantize_dynamic_flat_kernel(
     const Idx g = static_cast<Idx>(blockIdx.x) * kFlatThreads + tid;
     const Idx n_rounds = (nvec + chunk - 1) / chunk;
 
-    auto load_round = [&](Idx rd, BF16x16 (&v)[kFlatU]) {
+    // Phase 2 walks the rounds backwards, so the rounds phase 1 reads last are
+    // the ones it re-reads first: phase 1 loads those (up to kFlatKeepBytes)
+    // with an evict-last L2 policy so they are still in L2 for phase 2, which
+    // re-reads them with evict-first so they do not stay pinned after the
+    // kernel; every other load has the default policy.
+    const Idx keep_rounds = static_cast<Idx>(kFlatKeepBytes / (32 * static_cast<int64_t>(chunk)));
+    const uint64_t pol_keep = l2_policy_evict_last();
+    const uint64_t pol_done = l2_policy_evict_first();
+    auto load_round = [&](Idx rd, BF16x16 (&v)[kFlatU], int hint) {  // hint: 0 none, 1 keep, 2 done
 #pragma unroll
         for (int u = 0; u < kFlatU; ++u) {
             const Idx idx = rd * chunk + u * S + g;
-            if (idx < nvec) {
-                v[u] = ldg_32B(x + 32 * static_cast<int64_t>(idx), a32);
-            } else {
+            const uint8_t *p = x + 32 * static_cast<int64_t>(idx);
+            if (idx >= nvec) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k) v[u].w[k] = 0u;
+            } else if (hint == 0) {
+                v[u] = ldg_32B(p, a32);
+            } else {
+                v[u] = ldg_32B_policy(p, a32, hint == 1 ? pol_keep : pol_done);
             }
         }
     };
@@ -300,7 +351,7 @@ __global__ void __launch_bounds__(kFlatThreads, 2) quantize_dynamic_flat_kernel(
     uint32_t m = 0;
     BF16x16 v[kFlatU];
     for (Idx rd = 0; rd < n_rounds; ++rd) {
-        load_round(rd, v);
+        load_round(rd, v, rd + keep_rounds >= n_rounds ? 1 : 0);
 #pragma unroll
         for (int u = 0; u < kFlatU; ++u) m = max(m, absmax_bf16x16(v[u]));
     }
@@ -334,7 +385,7 @@ __global__ void __launch_bounds__(kFlatThreads, 2) quantize_dynamic_flat_kernel(
     // each group of 4 lanes (nvec and every warp's first index are multiples
     // of 4), so the scale gather's shuffles see consistent neighbours.
     for (Idx rd = n_rounds; rd-- > 0;) {
-        if (rd + 1 != n_rounds) load_round(rd, v);
+        if (rd + 1 != n_rounds) load_round(rd, v, rd + keep_rounds >= n_rounds ? 2 : 0);
 #pragma unroll
         for (int u = 0; u < kFlatU; ++u) {
             const Idx idx = rd * chunk + u * S + g;
