@@ -155,27 +155,112 @@ __device__ __forceinline__ void store_row(const GemmParams &p, const uint32_t (&
 #pragma unroll
     for (int q4 = 0; q4 < NC / 64; ++q4) {  // groups of 4 blocks (64 columns)
         uint32_t sf_word = 0;
+        uint32_t cw[8];  // the group's 32 bytes of codes
+        const int64_t nblk0 = (n0 >> 4) + 4 * q4;
+        uint8_t *qrow = p.yq + m * (p.N / 2) + nblk0 * 8;
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
             const int bi = 4 * q4 + b;  // block within the NC columns
-            const int64_t nblk = (n0 >> 4) + bi;
-            const bool ok_blk = row_ok && nblk < nb_y;
+            const bool ok_blk = row_ok && nblk0 + b < nb_y;
             const uint4 v0 = make_uint4(pk[8 * bi], pk[8 * bi + 1], pk[8 * bi + 2], pk[8 * bi + 3]);
             const uint4 v1 =
                 make_uint4(pk[8 * bi + 4], pk[8 * bi + 5], pk[8 * bi + 6], pk[8 * bi + 7]);
             const uint32_t mb = max(absmax_bf16x8(v0), absmax_bf16x8(v1));
             const BlockScale bs = block_scale(__uint_as_float(mb << 16), s_enc_y, inv_tab);
-            if (ok_blk) {
-                amax_bits = max(amax_bits, mb);
-                *reinterpret_cast<uint2 *>(p.yq + m * (p.N / 2) + nblk * 8) =
-                    make_uint2(quantize_bf16x8(v0, bs.inv), quantize_bf16x8(v1, bs.inv));
-            }
+            cw[2 * b] = quantize_bf16x8(v0, bs.inv);
+            cw[2 * b + 1] = quantize_bf16x8(v1, bs.inv);
+            if (ok_blk) amax_bits = max(amax_bits, mb);
             sf_word |= (ok_blk ? bs.sf : 0u) << (8 * b);
         }
-        const int64_t nblk0 = (n0 >> 4) + 4 * q4;
+        // One 32-byte store (a whole sector) when the four blocks are in range
+        // and the address is 32-byte aligned, else one 8-byte store per block.
+        if (row_ok && nblk0 + 3 < nb_y && (reinterpret_cast<uintptr_t>(qrow) & 31) == 0) {
+            stg256(qrow, cw[0], cw[1], cw[2], cw[3], cw[4], cw[5], cw[6], cw[7]);
+        } else {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                if (row_ok && nblk0 + b < nb_y)
+                    *reinterpret_cast<uint2 *>(qrow + 8 * b) = make_uint2(cw[2 * b], cw[2 * b + 1]);
+        }
         if (nblk0 < nb4_y * 4)
             *reinterpret_cast<uint32_t *>(p.ysf + sf_offset(m, nblk0, nb4_y)) = sf_word;
     }
+}
+
+// The epilogue of 64 accumulator columns (columns n0..n0+63 of row m) held
+// in registers as raw fp32 (r0: the first 32, r1: the next 32), one block of
+// 16 columns at a time: alpha, activation, bf16 rounding, the bf16 Y store
+// and the fused quantize of that block, so each block's registers are free
+// again before the next block starts (with the 64 raw values pinned in an
+// 80-register budget, converting all 64 columns first left no room for
+// independent work).  Same arithmetic per element, and the same outputs, as
+// cvt_32 on both halves followed by store_row<64>.
+template <bool kGelu>
+__device__ __forceinline__ void store_blocks_64(const GemmParams &p, const uint32_t (&r0)[32],
+                                                const uint32_t (&r1)[32], float alpha, int64_t m,
+                                                int64_t n0, float s_enc_y, const float *inv_tab,
+                                                uint32_t &amax_bits) {
+    const bool row_ok = m < p.M;
+    const bool want_y = row_ok && p.y != nullptr;
+    uint8_t *yrow = want_y ? p.y + (m * p.N + n0) * 2 : nullptr;
+    const bool y_fast = n0 + 64 <= p.N && (p.N & 15) == 0 &&
+                        (reinterpret_cast<uintptr_t>(p.y) & 31) == 0;
+    const int64_t rows_pad = (p.M + 127) & ~int64_t(127);
+    const bool want_q = p.yq != nullptr && m < rows_pad;
+    const int64_t nb_y = p.N / 16;
+    const int64_t nblk0 = n0 >> 4;
+    uint32_t cw[8];
+    uint32_t sf_word = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const uint32_t(&r)[32] = b < 2 ? r0 : r1;
+        const int base = (b & 1) * 16;
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float2 h = __fmul2_rn(make_float2(__uint_as_float(r[base + 2 * i]),
+                                              __uint_as_float(r[base + 2 * i + 1])),
+                                  splat2(alpha));
+            if (kGelu) h = gelu_erf2(h);
+            const __nv_bfloat162 bb = __floats2bfloat162_rn(h.x, h.y);
+            pk[i] = *reinterpret_cast<const uint32_t *>(&bb);
+        }
+        if (want_y) {
+            if (y_fast) {
+                stg256(yrow + 32 * b, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+            } else {
+                if (n0 + 16 * b < p.N)
+                    *reinterpret_cast<uint4 *>(yrow + 32 * b) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                if (n0 + 16 * b + 8 < p.N)
+                    *reinterpret_cast<uint4 *>(yrow + 32 * b + 16) =
+                        make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+        }
+        if (want_q) {
+            const bool ok_blk = row_ok && nblk0 + b < nb_y;
+            const uint4 v0 = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            const uint4 v1 = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            const uint32_t mb = max(absmax_bf16x8(v0), absmax_bf16x8(v1));
+            const BlockScale bs = block_scale(__uint_as_float(mb << 16), s_enc_y, inv_tab);
+            cw[2 * b] = quantize_bf16x8(v0, bs.inv);
+            cw[2 * b + 1] = quantize_bf16x8(v1, bs.inv);
+            if (ok_blk) amax_bits = max(amax_bits, mb);
+            sf_word |= (ok_blk ? bs.sf : 0u) << (8 * b);
+        }
+    }
+    if (!want_q) return;
+    uint8_t *qrow = p.yq + m * (p.N / 2) + nblk0 * 8;
+    if (row_ok && nblk0 + 3 < nb_y && (reinterpret_cast<uintptr_t>(qrow) & 31) == 0) {
+        stg256(qrow, cw[0], cw[1], cw[2], cw[3], cw[4], cw[5], cw[6], cw[7]);
+    } else {
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            if (row_ok && nblk0 + b < nb_y)
+                *reinterpret_cast<uint2 *>(qrow + 8 * b) = make_uint2(cw[2 * b], cw[2 * b + 1]);
+    }
+    const int64_t nb4_y = (nb_y + 3) / 4;
+    if (nblk0 < nb4_y * 4)
+        *reinterpret_cast<uint32_t *>(p.ysf + sf_offset(m, nblk0, nb4_y)) = sf_word;
 }
 
 // Warp-reduces the fused output's |Y| maximum and folds it into amax_y.

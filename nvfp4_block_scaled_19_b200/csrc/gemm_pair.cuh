@@ -386,8 +386,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty_l);
-                cvt_32<true>(r0, alpha, pk);
-                cvt_32<true>(r1, alpha, pk + 16);
+                store_blocks_64<true>(p, r0, r1, alpha, int64_t(tc.m_blk) * Cfg::BM + row_in_tile,
+                                      int64_t(tc.n_blk) * Cfg::BN + col0, s_enc_y, inv_tab,
+                                      amax_bits);
+                continue;
             } else {
                 drain_cols<Cfg::EPI_COLS, kGelu>(taddr, alpha, pk);
                 tc_fence_before();
