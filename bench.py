@@ -653,34 +653,42 @@ def host_e2e(nv, layers, args, device, dist, world) -> dict:
     """Same metric end to end: pinned host X in, host Y out, copies timed.
     Independent layers go through nvfp4_linear_host; a chain (a layer fed by
     the previous layer's fused output) through the Python API, copying every
-    drawn X in and the last layer's Y out."""
+    drawn X in and the last layer's Y out.  Each independent layer runs on a
+    stream of its own (with its own workspaces), so one layer's host-to-device
+    copy can overlap another's device-to-host copy and compute; a layer's
+    steps stay in order on its stream."""
     if any(L.spec.x_from_prev or L.row_scales or L.fp8 or L.stale or L.sharded for L in layers):
         return chain_e2e(nv, layers, args, device, dist, world)
-    stream = torch.cuda.current_stream()
+    main = torch.cuda.current_stream()
     hosts = []
     for L in layers:
         xh = L.x_cpu.contiguous().pin_memory()
         yh = torch.empty(L.M, L.N, dtype=torch.bfloat16).pin_memory()
-        hosts.append((xh, yh, L.lin.host_workspace(L.M, device)))
+        hosts.append((xh, yh, L.lin.host_workspace(L.M, device), torch.cuda.Stream(device)))
     steps = max(1, min(args.steps, args.e2e_steps))
     for _ in range(2):
-        for L, (xh, yh, ws) in zip(layers, hosts):
-            L.lin.forward_host(xh, yh, ws)
+        for L, (xh, yh, ws, st) in zip(layers, hosts):
+            L.lin.forward_host(xh, yh, ws, stream=st)
     torch.cuda.synchronize()
     barrier(dist, device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(main)
+    for _, _, _, st in hosts:
+        st.wait_event(e0)
     for _ in range(steps):
-        for L, (xh, yh, ws) in zip(layers, hosts):
-            L.lin.forward_host(xh, yh, ws)
-    e1.record(stream)
+        for L, (xh, yh, ws, st) in zip(layers, hosts):
+            L.lin.forward_host(xh, yh, ws, stream=st)
+    for _, _, _, st in hosts:
+        main.wait_stream(st)
+    e1.record(main)
     torch.cuda.synchronize()
     sec = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, device)
     flops = sum(L.flops for L in layers) * steps
     return {"value": round(aggregate(flops, world, sec) / 1e12, 3), "unit": UNIT,
             "h2d_bytes_per_step": sum(L.M * L.K * 2 for L in layers),
             "d2h_bytes_per_step": sum(L.M * L.N * 2 for L in layers),
-            "steps": steps, "api": "nvfp4_linear_host (C ABI, pinned host buffers)"}
+            "steps": steps, "api": "nvfp4_linear_host (C ABI, pinned host buffers; "
+                                   "one stream per independent layer)"}
 
 
 def chain_e2e(nv, layers, args, device, dist, world) -> dict:

@@ -375,18 +375,25 @@ class NVFP4Linear:
         single_launch=False passes no dynamic-quantize workspace, so the call
         quantizes X with nvfp4_tensor_amax + nvfp4_quantize."""
         M = x_host.shape[0]
+        dyn = ws.get("dyn")
+        if dyn is None:
+            dyn = dynamic_workspace(ws["x"].device)
         w = LinearWorkspace(ws["x"].data_ptr(), ws["xq"].data_ptr(), ws["xsf"].data_ptr(),
                             ws["amax"].data_ptr(), ws["s_dec"].data_ptr(), ws["y"].data_ptr(),
-                            dynamic_workspace(ws["x"].device).data_ptr() if single_launch
-                            else None)
+                            dyn.data_ptr() if single_launch else None)
         _check("nvfp4_linear_host", lib().nvfp4_linear_host(
             x_host.data_ptr(), M, self.K, self.w.q.data_ptr(), self.w.sf.data_ptr(),
             self.w.s_dec.data_ptr(), self.N, y_host.data_ptr(), ctypes.byref(w),
             _stream(stream)))
 
     def host_workspace(self, M: int, device=None) -> dict:
+        """Device buffers for forward_host, including a dynamic-quantize
+        workspace of its own, so calls with different workspaces may run on
+        different streams at the same time."""
         dev = torch.device("cuda") if device is None else device
-        return {"x": torch.empty(M, self.K, dtype=torch.bfloat16, device=dev),
+        n = int(lib().nvfp4_quantize_dynamic_workspace_bytes())
+        return {"dyn": torch.zeros((n + 15) // 16 * 16, dtype=torch.uint8, device=dev),
+                "x": torch.empty(M, self.K, dtype=torch.bfloat16, device=dev),
                 "xq": torch.empty(M, self.K // 2, dtype=torch.uint8, device=dev),
                 "xsf": torch.empty(sf_bytes(M, self.K), dtype=torch.uint8, device=dev),
                 "amax": torch.empty(1, dtype=torch.float32, device=dev),
