@@ -53,6 +53,7 @@ SUSTAINED_AFTER_S = 0.5
 FP4_PER_BF16 = 4.0      # nominal dense FP4 / dense BF16 (9 / 2.25 PFLOP/s)
 FP8_PER_BF16 = 2.0      # nominal dense FP8 / dense BF16 (4.5 / 2.25 PFLOP/s)
 NOMINAL_FP4_TFLOPS = 9000.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, vendor figure
 
 
 GEMM_SOURCES = ["gemm.h", "gemm.cu", "gemm_pair.cuh", "gemm_common.cuh", "ptx.cuh",
@@ -563,6 +564,7 @@ def gpu_arm(args) -> dict | None:
          "of_nominal_4_5pf": round(value / world / (NOMINAL_FP4_TFLOPS / 2), 4),
          "regime": regime},
         "quantize": {"gbs": round(q_gbs, 1), "pct_hbm": round(q_gbs / hbm, 4),
+                     "pct_hbm_nominal_8tbs": round(q_gbs / NOMINAL_HBM_GBS, 4),
                      "ms_per_step": round(q_ms_sum, 5),
                      "note": ("per-token quantize, one pass: algorithmic bytes 2.5625 B/elem "
                               "+ per-row scales" if row else
@@ -842,7 +844,8 @@ def quantize_sweep(args) -> dict:
             torch.cuda.synchronize()
             us = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev) * 1e3
             gbs = n * bpe / (us * 1e-6) / 1e9
-            row[name] = {"us": round(us, 2), "gbs": round(gbs, 1), "pct_hbm": round(gbs / hbm, 4)}
+            row[name] = {"us": round(us, 2), "gbs": round(gbs, 1), "pct_hbm": round(gbs / hbm, 4),
+                         "pct_hbm_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4)}
         rows_out.append(row)
         del x, out
     code, detail = nv.device_error()
