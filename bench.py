@@ -494,9 +494,7 @@ def gpu_arm(args) -> dict | None:
     bf16_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     bf16_sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     per_bf16 = FP8_PER_BF16 if fp8 else FP4_PER_BF16
-    sustained = total_s >= SUSTAINED_AFTER_S
-    regime = "sustained" if sustained else "burst"
-    fp4_peak = per_bf16 * (bf16_sust if sustained else bf16_burst)
+    fp4_peak, regime, peak_note = tensor_peak(per_bf16, bf16_burst, bf16_sust, total_s)
     gemm_tflops = layers[top].flops / (g_avg[top] * 1e-3) / 1e12
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     q_bytes = sum(L.quant_bytes for L in layers)
@@ -583,15 +581,7 @@ def gpu_arm(args) -> dict | None:
                      "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
                      "traffic": traffic, "traffic_source": traffic_src,
                      "algorithmic_bytes": layers[top].gemm_bytes,
-                     "peak_source": (f"{peak_src}: {per_bf16:g} x bf16_tflops_sustained "
-                                     f"({bf16_sust}): the timed steps ran {total_s:.2f} s back "
-                                     f"to back (>= {SUSTAINED_AFTER_S} s: at the power cap); "
-                                     f"burst would be {per_bf16 * bf16_burst:.1f}")
-                                    if sustained else
-                                    (f"{peak_src}: {per_bf16:g} x bf16_tflops burst "
-                                     f"({bf16_burst}): the timed steps ran {total_s:.3f} s "
-                                     f"(< {SUSTAINED_AFTER_S} s); sustained would be "
-                                     f"{per_bf16 * bf16_sust:.1f}")},
+                     "peak_source": f"{peak_src}: {peak_note}"},
         "clocks": clocks,
         "graph": graph,
         "e2e": e2e,
@@ -618,6 +608,24 @@ def timed_steps(nv, layers, flush, steps):
     q_ms = [[ev[s][i][0].elapsed_time(ev[s][i][1]) for s in range(steps)] for i in range(n_l)]
     g_ms = [[ev[s][i][1].elapsed_time(ev[s][i][2]) for s in range(steps)] for i in range(n_l)]
     return q_ms, g_ms
+
+
+def tensor_peak(per_bf16: float, bf16_burst: float, bf16_sust: float,
+                timed_s: float) -> tuple[float, str, str]:
+    """The tensor roofline for a run whose timed steps took timed_s seconds of
+    device time back to back: per_bf16 x the burst bf16 figure for a short
+    run, x the sustained one from SUSTAINED_AFTER_S on (the GPU then sits at
+    its power cap, where the sustained figure was measured).  Returns (peak
+    TFLOP/s, "burst" | "sustained", a note naming the figure)."""
+    if timed_s >= SUSTAINED_AFTER_S:
+        return (per_bf16 * bf16_sust, "sustained",
+                f"{per_bf16:g} x bf16_tflops_sustained ({bf16_sust}): the timed steps ran "
+                f"{timed_s:.2f} s back to back (>= {SUSTAINED_AFTER_S} s, at the power cap); "
+                f"burst would be {per_bf16 * bf16_burst:.1f}")
+    return (per_bf16 * bf16_burst, "burst",
+            f"{per_bf16:g} x bf16_tflops burst ({bf16_burst}): the timed steps ran "
+            f"{timed_s:.3f} s (< {SUSTAINED_AFTER_S} s); sustained would be "
+            f"{per_bf16 * bf16_sust:.1f}")
 
 
 def ffn_down_modes(nv, args, flush, device, fp4_peak) -> dict:

@@ -46,6 +46,9 @@ def test_gpu_arm_line():
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert 0 < r["frac"] < 1.5 and abs(r["achieved"] / r["peak"] - r["frac"]) < 1e-3
     assert r["traffic"] is None or r["traffic"] > 0
+    # 20 steps of ~0.8 ms: a short run, measured against the burst figure.
+    assert d["pct_fp4_peak"]["regime"] == "burst" and "burst (" in r["peak_source"]
+    assert abs(d["pct_fp4_peak"]["of_4x_measured_bf16_burst"] * r["peak"] - d["value"]) < 1.0
     e = d["e2e"]
     assert e["h2d_bytes_per_step"] == 2 * M * (H + F)
     assert e["d2h_bytes_per_step"] == 2 * M * (F + H)
@@ -83,6 +86,18 @@ def test_job_flops_replicas_and_shards():
     assert bench.job_flops(shards, 4) == 2 * 4608 * 9216 * 3072
     one = [_L(4608, 9216, 3072, m_global=4608, sharded=True)]
     assert bench.job_flops(one, 1) == 2 * 4608 * 9216 * 3072
+
+
+def test_tensor_peak_follows_the_timed_length():
+    # Pool measurements: bf16 1627.8 burst, 1395 sustained; FP4 = 4 x bf16.
+    import bench
+    short = bench.tensor_peak(4.0, 1627.8, 1395.0, 0.016)
+    long = bench.tensor_peak(4.0, 1627.8, 1395.0, 1.6)
+    assert short[:2] == (4.0 * 1627.8, "burst")
+    assert long[:2] == (4.0 * 1395.0, "sustained")
+    edge = bench.tensor_peak(2.0, 1627.8, 1395.0, bench.SUSTAINED_AFTER_S)
+    assert edge[:2] == (2.0 * 1395.0, "sustained")
+    assert "burst would be" in long[2] and "sustained would be" in short[2]
 
 
 @pytest.mark.gpu
