@@ -807,8 +807,20 @@ def cpu_baseline(w, target_s: float) -> dict:
         s, f, desc = oracle_sample(w, rows)
         secs, flops, passes = secs + s, flops + f, passes + 1
     return {"value": round(flops / secs / 1e12, 6), "unit": UNIT,
-            "cores": oracle.num_threads(), "kind": "oracle",
+            "cores": oracle.num_threads(), "cpu_model": cpu_model(), "kind": "oracle",
             "sample": f"{passes} passes of: {desc}", "seconds": round(secs, 3)}
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def quantize_sweep(args) -> dict:
@@ -891,7 +903,7 @@ def reference_arm(args) -> dict | None:
             "data": "synthetic", "config": {"workload": w.name, "M": w.M,
                                             "layers": [[l.name, l.K, l.N] for l in w.layers]},
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores,
-                             "kind": "oracle", "sample": desc},
+                             "cpu_model": cpu_model(), "kind": "oracle", "sample": desc},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
