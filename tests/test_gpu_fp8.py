@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_common import TOL, require_cuda
+from gpu_common import TOL, bf16_from_fp64, check_fused_blocks, require_cuda
 from workloads import WORKLOADS, bf16_bits, draw_w, draw_x, layer_inputs
 
 pytestmark = pytest.mark.gpu
@@ -105,3 +105,34 @@ def test_quantize_fp8_empty(nv):
     oq, os_dec, _ = oracle.quantize_fp8(bf16_bits(x), 0, 64)
     assert q.size == 0 and oq.size == 0
     assert s_dec == os_dec
+
+
+@pytest.mark.parametrize("act", ["none", "gelu"])
+@pytest.mark.parametrize("M,N,K", [(256, 256, 32), (300, 512, 96), (1000, 768, 3072)])
+def test_gemm_fp8_fused_nvfp4_output(nv, orc, M, N, K, act):
+    """The FP8 GEMM's fused epilogue, as for the NVFP4 GEMM: bf16 Y (after
+    GELU when asked), the next layer's NVFP4 codes and scales with a static
+    S_enc, amax of Y and its decode scale.  The oracle computes the FP8 layer
+    in fp64, applies its own GELU, rounds to bf16 and quantizes."""
+    x = draw_x("lognormal_channels", M, K, seed=3 * M + K, index=0)
+    w = draw_w(N, K, None, seed=3 * M + K, index=1)
+    ref = _oracle_fp8_linear(x, w)
+    out_ref = oracle.gelu(ref) if act == "gelu" else ref
+    s_enc_y = float(np.float32(2688.0) / np.float32(1.25 * np.abs(out_ref).max()))
+    lin = nv.FP8Linear(w.cuda())
+    fq = nv.FusedQuant(torch.tensor([s_enc_y], dtype=torch.float32, device="cuda"),
+                       nv.empty_nvfp4(M, N), torch.zeros(1, dtype=torch.float32, device="cuda"),
+                       nv.ACT_GELU if act == "gelu" else nv.ACT_NONE)
+    y = lin(x.cuda(), fused=fq)
+    torch.cuda.synchronize()
+    code, detail = nv.device_error()
+    assert code == 0, f"device wait timed out (tag {detail})"
+    yg = y.float().cpu().numpy()
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    slope = 1.13 if act == "gelu" else 1.0                  # GELU's slope is at most 1.129
+    err = np.abs(yg.astype(np.float64) - out_ref)
+    assert np.all(err <= slope * TOL * (np.abs(ref) + rms)), f"{M}x{N}x{K} {act} Y"
+    check_fused_blocks(orc, yg, bf16_from_fp64(out_ref), fq.out.q.cpu().numpy(),
+                       fq.out.sf.cpu().numpy(), np.arange(M), s_enc_y, f"fp8 {M}x{N}x{K} {act}")
+    assert np.float32(fq.amax.item()) == np.float32(np.abs(yg).max())
+    assert np.float32(fq.out.s_dec.item()) == np.float32(1.0) / np.float32(s_enc_y)
