@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_common import TOL, require_cuda
+from gpu_common import TOL, bf16_from_fp64, check_fused_blocks, require_cuda
 from workloads import WORKLOADS, bf16_bits, draw_w, draw_x, layer_inputs
 
 pytestmark = pytest.mark.gpu
@@ -102,3 +102,39 @@ def test_quantize_rowwise_empty(nv):
     """0 rows: nothing to quantize and no per-row scales; the call succeeds."""
     x = torch.zeros(0, 64, dtype=torch.bfloat16)
     _assert_equal(_gpu_rowwise(nv, x), oracle.quantize_rowwise(bf16_bits(x), 0, 64), "0x64")
+
+
+@pytest.mark.parametrize("act", ["none", "gelu"])
+@pytest.mark.parametrize("M,N,K", [(256, 512, 512), (130, 208, 128), (300, 512, 576)])
+def test_gemm_rowscale_fused(nv, orc, M, N, K, act):
+    """Per-row decode scales of A with the fused next-layer NVFP4 quantize
+    (plain and GELU): the epilogue's alpha is per row; Y, codes, scales, amax
+    and decode scale as for the per-tensor GEMM's fused epilogue."""
+    x = draw_x("lognormal_channels", M, K, seed=2 * M + N, index=0).float()
+    x *= torch.exp(torch.linspace(-1.0, 1.0, M))[:, None]       # rows of different scale
+    x = x.to(torch.bfloat16)
+    w = draw_w(N, K, None, seed=2 * M + N, index=1)
+    aq, asf, asd, _ = oracle.quantize_rowwise(bf16_bits(x), M, K)
+    bq, bsf, bsd, _ = oracle.quantize_dynamic(bf16_bits(w), N, K)
+    ref = oracle.gemm_rowwise(aq, asf, asd, bq, bsf, bsd, M, N, K)
+    out_ref = oracle.gelu(ref) if act == "gelu" else ref
+    s_enc_y = float(np.float32(2688.0) / np.float32(1.25 * np.abs(out_ref).max()))
+    lin = nv.NVFP4Linear(w.cuda())
+    fq = nv.FusedQuant(torch.tensor([s_enc_y], dtype=torch.float32, device="cuda"),
+                       nv.empty_nvfp4(M, N), torch.zeros(1, dtype=torch.float32, device="cuda"),
+                       nv.ACT_GELU if act == "gelu" else nv.ACT_NONE)
+    y = nv.gemm(nv.quantize_rowwise(x.cuda()), lin.w, fused=fq)
+    torch.cuda.synchronize()
+    code, detail = nv.device_error()
+    assert code == 0, f"device wait timed out (tag {detail})"
+    yg = y.float().cpu().numpy()
+    slope = 1.13 if act == "gelu" else 1.0                  # GELU's slope is at most 1.129
+    for m in range(M):
+        rms = float(np.sqrt(np.mean(ref[m] * ref[m])))
+        err = np.abs(yg[m].astype(np.float64) - out_ref[m])
+        assert np.all(err <= slope * TOL * (np.abs(ref[m]) + rms)), f"{M}x{N}x{K} {act} row {m}"
+    check_fused_blocks(orc, yg, bf16_from_fp64(out_ref), fq.out.q.cpu().numpy(),
+                       fq.out.sf.cpu().numpy(), np.arange(M), s_enc_y,
+                       f"rowscale {M}x{N}x{K} {act}")
+    assert np.float32(fq.amax.item()) == np.float32(np.abs(yg).max())
+    assert np.float32(fq.out.s_dec.item()) == np.float32(1.0) / np.float32(s_enc_y)
