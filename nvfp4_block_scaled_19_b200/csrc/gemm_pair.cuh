@@ -37,6 +37,8 @@
 // single `full` barrier and the fully unrolled stage body.
 #pragma once
 
+#include <type_traits>
+
 namespace nvfp4 {
 
 template <int STAGES_, int EPI_WARPS_>
@@ -241,30 +243,68 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Cfg::THREADS, 1)
             uint32_t phase = 0;
             bool ok = true;
             int local = 0;
+            const uint32_t full_a = smem_addr(full);
+            const uint32_t empty_a = smem_addr(empty);
+            const uint32_t sf_t0 = tmem_base + Cfg::SF_BASE;
+            // One full 256-element stage in ring slot S: wait, four MMAs, one
+            // commit.  S is a compile-time constant, so every address and
+            // descriptor here is a constant offset from a register.
+            auto full_stage = [&](auto slot, uint32_t acc0) -> bool {
+                constexpr int S = decltype(slot)::value;
+                if (!mbar_wait_at(full_a + 8 * S, phase, abort_flag, 13)) return false;
+                tc_fence_after();
+                const uint64_t adesc = adesc0 + ((uint64_t(S) * Cfg::A_BYTES) >> 4);
+                const uint64_t bdesc = bdesc0 + ((uint64_t(S) * Cfg::B_BYTES) >> 4);
+                const uint32_t sfa_t = sf_t0 + S * Cfg::SLOT_COLS;
+                const uint32_t sfb_t = sfa_t + Cfg::SFA_COLS;
+                mma(adesc, bdesc, sfa_t, sfb_t, 0, acc0);
+#pragma unroll
+                for (int j = 1; j < 4; ++j) mma(adesc, bdesc, sfa_t, sfb_t, j, 1u);
+                tc_commit_pair_at(empty_a + 8 * S, 0x3);
+                return true;
+            };
             for (int t = pair; t < num_tiles && ok; t += n_pairs, ++local) {
                 if (!mbar_wait(acc_empty, (local & 1) ^ 1, abort_flag, 12)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                // Full 256-element stages: one wait, four MMAs, one commit.
-                for (int ks = 0; ks < k_full; ++ks) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag, 13)) {
+                // Full 256-element stages, unrolled over the ring and entered
+                // at the current slot.
+                static_assert(Cfg::STAGES == 5, "the stage loop is unrolled over 5 slots");
+                int ks = 0;
+                auto step = [&](auto slot) -> bool {
+                    constexpr int S = decltype(slot)::value;
+                    if (ks == k_full) return false;
+                    if (!full_stage(slot, ks > 0 ? 1u : 0u)) {
                         ok = false;
-                        break;
+                        return false;
                     }
-                    tc_fence_after();
-                    const uint64_t adesc = adesc0 + static_cast<uint64_t>((stage * Cfg::A_BYTES) >> 4);
-                    const uint64_t bdesc = bdesc0 + static_cast<uint64_t>((stage * Cfg::B_BYTES) >> 4);
-                    const uint32_t sfa_t = tmem_base + Cfg::SF_BASE + stage * Cfg::SLOT_COLS;
-                    const uint32_t sfb_t = sfa_t + Cfg::SFA_COLS;
-                    mma(adesc, bdesc, sfa_t, sfb_t, 0, ks > 0 ? 1u : 0u);
-#pragma unroll
-                    for (int j = 1; j < 4; ++j) mma(adesc, bdesc, sfa_t, sfb_t, j, 1u);
-                    tc_commit_pair(&empty[stage], 0x3);
-                    if (++stage == Cfg::STAGES) {
+                    ++ks;
+                    if constexpr (S + 1 == Cfg::STAGES) {
                         stage = 0;
                         phase ^= 1;
+                    } else {
+                        stage = S + 1;
+                    }
+                    return true;
+                };
+                while (ok && ks < k_full) {
+                    switch (stage) {
+                        case 0:
+                            if (!step(std::integral_constant<int, 0>{})) break;
+                            [[fallthrough]];
+                        case 1:
+                            if (!step(std::integral_constant<int, 1>{})) break;
+                            [[fallthrough]];
+                        case 2:
+                            if (!step(std::integral_constant<int, 2>{})) break;
+                            [[fallthrough]];
+                        case 3:
+                            if (!step(std::integral_constant<int, 3>{})) break;
+                            [[fallthrough]];
+                        default:
+                            step(std::integral_constant<int, 4>{});
                     }
                 }
                 if (ok && k_tail > 0) {

@@ -75,9 +75,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Waits for the phase with the given parity to complete.  Gives up (and
 // returns false) when *abort is set by another thread of the CTA, or after
 // timeout_ns, in which case it records the timeout and sets *abort.
-__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                              int tag, uint64_t timeout_ns) {
-    const uint32_t a = smem_addr(bar);
+__device__ __forceinline__ bool mbar_wait_for_at(uint32_t a, uint32_t parity, volatile int *abort,
+                                                 int tag, uint64_t timeout_ns) {
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
@@ -91,9 +90,20 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, vo
     }
 }
 
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                              int tag, uint64_t timeout_ns) {
+    return mbar_wait_for_at(smem_addr(bar), parity, abort, tag, timeout_ns);
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           int tag) {
     return mbar_wait_for(bar, parity, abort, tag, kWaitTimeoutNs);
+}
+
+// mbar_wait on a barrier given by its shared-memory address.
+__device__ __forceinline__ bool mbar_wait_at(uint32_t a, uint32_t parity, volatile int *abort,
+                                             int tag) {
+    return mbar_wait_for_at(a, parity, abort, tag, kWaitTimeoutNs);
 }
 
 // Warp-uniform wait: lane 0 polls, every lane gets the same answer, so a
@@ -295,12 +305,16 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 
 // Arrives once on the barrier at this offset in every CTA of `cta_mask`
 // when all tcgen05 operations issued so far by this thread have completed.
-__device__ __forceinline__ void tc_commit_pair(uint64_t *bar, uint16_t cta_mask) {
+__device__ __forceinline__ void tc_commit_pair_at(uint32_t bar_a, uint16_t cta_mask) {
     asm volatile(
         "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-        " [%0], %1;" ::"r"(smem_addr(bar)),
+        " [%0], %1;" ::"r"(bar_a),
         "h"(cta_mask)
         : "memory");
+}
+
+__device__ __forceinline__ void tc_commit_pair(uint64_t *bar, uint16_t cta_mask) {
+    tc_commit_pair_at(smem_addr(bar), cta_mask);
 }
 
 __device__ __forceinline__ void mma_mxf4nvf4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
