@@ -54,10 +54,13 @@ __device__ __forceinline__ void mbar_arrive_relaxed(uint64_t *bar) {
                  : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-                 "r"(bytes)
+__device__ __forceinline__ void mbar_arrive_expect_tx_at(uint32_t bar_a, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_a), "r"(bytes)
                  : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    mbar_arrive_expect_tx_at(smem_addr(bar), bytes);
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
@@ -108,11 +111,16 @@ __device__ __forceinline__ bool mbar_wait_at(uint32_t a, uint32_t parity, volati
 
 // Warp-uniform wait: lane 0 polls, every lane gets the same answer, so a
 // timeout can never split the warp before a .sync.aligned instruction.
+__device__ __forceinline__ bool mbar_wait_warp_at(uint32_t a, uint32_t parity, volatile int *abort,
+                                                  int tag) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_at(a, parity, abort, tag) ? 1 : 0;
+    return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort,
                                                int tag) {
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, tag) ? 1 : 0;
-    return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+    return mbar_wait_warp_at(smem_addr(bar), parity, abort, tag);
 }
 
 // Drain wait used only on the abort path: bounded, never sets flags.
@@ -184,24 +192,34 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap *m, uint64_t *bar,
 // 2-D tiled TMA load for a CTA pair: data lands in this CTA's shared memory,
 // completion bytes are counted on the barrier at `bar_cluster` (a
 // shared::cluster address, normally the pair leader's).  No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *m, uint32_t bar_cluster, void *dst,
-                                                 int x, int y, uint64_t policy) {
+__device__ __forceinline__ void tma_load_2d_pair_at(const CUtensorMap *m, uint32_t bar_cluster,
+                                                    uint32_t dst_a, int x, int y, uint64_t policy) {
     asm volatile(
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_addr(dst)),
+        ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst_a),
         "l"(m), "r"(bar_cluster), "r"(x), "r"(y), "l"(policy)
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *m, uint32_t bar_cluster, void *dst,
+                                                 int x, int y, uint64_t policy) {
+    tma_load_2d_pair_at(m, bar_cluster, smem_addr(dst), x, y, policy);
+}
+
 // 3-D tiled TMA load into this CTA's shared memory, completion on `bar`.
 // No multicast.
-__device__ __forceinline__ void tma_load_3d(const CUtensorMap *m, uint64_t *bar, void *dst, int x,
-                                            int y, int z, uint64_t policy) {
+__device__ __forceinline__ void tma_load_3d_at(const CUtensorMap *m, uint32_t bar_a, uint32_t dst_a,
+                                               int x, int y, int z, uint64_t policy) {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_addr(dst)),
-        "l"(m), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst_a),
+        "l"(m), "r"(bar_a), "r"(x), "r"(y), "r"(z), "l"(policy)
         : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(const CUtensorMap *m, uint64_t *bar, void *dst, int x,
+                                            int y, int z, uint64_t policy) {
+    tma_load_3d_at(m, smem_addr(bar), smem_addr(dst), x, y, z, policy);
 }
 
 // 2-D tiled TMA store from shared memory (bulk-group completion).
